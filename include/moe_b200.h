@@ -1,0 +1,210 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) DeepSeekMoE layer forward.
+ *
+ * The layer (a DeepSeekMoE feed-forward block, as listed step by step on the
+ * "DeepSeek-V3.2-Exp · Mixture of experts" page, section "All 19 steps"):
+ *
+ *   router    z = x W_r^T            one logit per routed expert
+ *             s = softmax(z) | sigmoid(z)
+ *             selection: top_k of s + b, restricted to the topk_groups best
+ *             of n_groups contiguous expert groups ("top-8 of s+b within the
+ *             top 4 groups"); b only steers the selection
+ *             gates G = route_scale * s / sum(s over the selection)  (normalize)
+ *                   G = route_scale * s                             (otherwise,
+ *             the GShard router of the "DeepSeekMoE" walkthrough, Step 2)
+ *   experts   E_e(x) = W2_e (silu(W1_e x) * (W3_e x))      fine-grained SwiGLU
+ *   shared    y_shared = Ws2 (silu(Ws1 x) * (Ws3 x))       always on, ungated
+ *   output    y = sum_e G_e E_e(x) + y_shared              (no residual)
+ *
+ * Tokens are one flattened axis of T rows (batch and positions folded
+ * together, as the page's quoted MoE.forward does). No token is dropped and
+ * no expert has a capacity limit.
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are dense row-major in device memory (HBM), element type
+ *     cfg->dtype (fp32 or bf16) unless stated; every base pointer must be
+ *     16-byte aligned; d and d_ff must be multiples of 8.
+ *   - The caller owns every buffer. The library allocates no device memory:
+ *     scratch lives in a caller-provided workspace of moe_workspace_size()
+ *     bytes (256-byte aligned).
+ *   - cfg is read on the host during the call only.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising. Results are ready
+ *     when the stream has drained.
+ *   - Errors are returned as moe_status values; nothing is thrown across the
+ *     ABI. Launch failures return MOE_ERR_CUDA, and the CUDA error code is
+ *     kept per host thread for moe_last_cuda_error(). Failures detected on the
+ *     device (a pipeline wait that timed out, an out-of-range expert index)
+ *     are recorded in a status word inside the workspace; read it with
+ *     moe_device_status().
+ *   - T == 0 is a valid no-op returning MOE_OK.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* bad cfg, null or misaligned pointer, negative T */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid layer outside what this build implements */
+  MOE_ERR_WORKSPACE = 3,    /* workspace null or smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+  MOE_ERR_DEVICE = 5        /* moe_device_status() found a device-side failure */
+} moe_status;
+
+enum { MOE_F32 = 0, MOE_BF16 = 1 };                 /* moe_cfg.dtype */
+enum { MOE_SOFTMAX = 0, MOE_SIGMOID = 1 };          /* moe_cfg.score_fn */
+enum { MOE_GROUP_TOP2_SUM = 0, MOE_GROUP_MAX = 1 }; /* moe_cfg.group_score */
+
+/* Device-status bits (moe_device_status). */
+enum {
+  MOE_DEV_WAIT_TIMEOUT = 1u << 0,   /* a bounded pipeline wait gave up */
+  MOE_DEV_BAD_EXPERT = 1u << 1,     /* an expert index outside [0, n_routed) */
+  MOE_DEV_DUP_EXPERT = 1u << 2,     /* a token lists the same expert twice */
+  MOE_DEV_TMEM_ALLOC = 1u << 3      /* tensor-memory allocation returned no columns */
+};
+
+/*
+ * Layer configuration. Field names follow the page's model arguments
+ * (dim, moe_inter_dim, n_routed_experts, n_shared_experts,
+ * n_activated_experts) and the router steps.
+ *   d            model dimension (dim)
+ *   d_ff         width of one routed expert (moe_inter_dim)
+ *   n_routed     N, routed experts (1..512)
+ *   n_shared     shared experts, fused into one MLP of width n_shared*d_ff
+ *   top_k        experts selected per token (1..16, <= topk_groups*N/n_groups)
+ *   n_groups     expert groups (1 = no group limit); must divide n_routed
+ *   topk_groups  groups kept per token (1..n_groups)
+ *   score_fn     MOE_SOFTMAX or MOE_SIGMOID
+ *   normalize    nonzero: gates normalised over the selection, then scaled
+ *   route_scale  gate multiplier (2.5 for the DeepSeek-V3 layer, 1 for GShard)
+ *   group_score  how a group is scored for the group limit: the sum of its
+ *                two largest s+b (MOE_GROUP_TOP2_SUM) or its largest (MOE_GROUP_MAX)
+ *   dtype        MOE_F32 (SIMT fp32 path) or MOE_BF16 (tensor-core path)
+ */
+typedef struct moe_cfg {
+  int32_t d;
+  int32_t d_ff;
+  int32_t n_routed;
+  int32_t n_shared;
+  int32_t top_k;
+  int32_t n_groups;
+  int32_t topk_groups;
+  int32_t score_fn;
+  int32_t normalize;
+  float route_scale;
+  int32_t group_score;
+  int32_t dtype;
+} moe_cfg;
+
+/*
+ * Bytes of device workspace that moe_route, moe_dispatch and moe_forward
+ * need for T tokens. Returns MOE_ERR_INVALID_ARG for an invalid cfg or
+ * T < 0, MOE_ERR_UNSUPPORTED outside the implemented range.
+ */
+MOE_API moe_status moe_workspace_size(const moe_cfg* cfg, int64_t T, size_t* bytes);
+
+/*
+ * Router only (the "Router:" steps of the equation list).
+ *   x        [T, d]      tokens, cfg->dtype
+ *   W_r      [N, d]      one router row per routed expert, cfg->dtype
+ *   b        [N] fp32    selection bias, or NULL for none
+ *   topk_idx [T, top_k] int32 out: selected experts, slots in descending s+b
+ *   gates    [T, top_k] fp32  out: gate of each slot (from the unbiased s)
+ * Logits are accumulated in fp32 with fp64 partial-sum carries; selection
+ * breaks exact ties toward the lower group / expert index.
+ */
+MOE_API moe_status moe_route(const moe_cfg* cfg, int64_t T, const void* x, const void* W_r, const float* b,
+                     int32_t* topk_idx, float* gates, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Expert histogram and expert-contiguous token lists (the quoted forward's
+ * bincount over the selected indices and its per-expert token lists).
+ *   topk_idx [T, top_k] int32 in (as written by moe_route)
+ *   counts   [N] int32 out: (token, slot) pairs per expert
+ *   offsets  [N+1] int32 out: exclusive prefix sum of counts
+ *   perm     [T*top_k] int32 out: perm[offsets[e] + r] = t*top_k + slot of
+ *            the r-th pair that chose e, tokens ascending (bit-exact, no
+ *            order-dependent atomics)
+ * Any output pointer may be NULL to skip copying it out. An index outside
+ * [0, N) or a repeated expert within one token sets a device-status bit.
+ */
+MOE_API moe_status moe_dispatch(const moe_cfg* cfg, int64_t T, const int32_t* topk_idx, int32_t* counts,
+                        int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The whole layer forward: y = Delta_ffn.
+ *   x            [T, d]
+ *   W_r, b       as for moe_route
+ *   W1, W3       [N, d_ff, d]        routed experts, stacked (out x in)
+ *   W2           [N, d, d_ff]
+ *   Ws1, Ws3     [n_shared*d_ff, d]  fused shared MLP; NULL iff n_shared == 0
+ *   Ws2          [d, n_shared*d_ff]
+ *   y            [T, d] out, cfg->dtype (fp32 accumulation, one rounding)
+ *   topk_idx_out, gates_out  optional [T, top_k] copies of the routing (NULL to skip)
+ * bf16 path: expert matmuls on tcgen05 tensor cores (bf16 x bf16 -> fp32),
+ * SwiGLU output and gated expert rows rounded to bf16, combine in fp32 in
+ * ascending expert order. fp32 path: the same steps on CUDA cores in fp32.
+ * Deterministic: two calls on the same inputs give the same bits.
+ */
+MOE_API moe_status moe_forward(const moe_cfg* cfg, int64_t T, const void* x, const void* W_r, const float* b,
+                       const void* W1, const void* W3, const void* W2, const void* Ws1,
+                       const void* Ws3, const void* Ws2, void* y, int32_t* topk_idx_out,
+                       float* gates_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_forward with the token rows in host memory: copies x_host [T, d] to
+ * the device inside the workspace, runs the layer, and copies y back to
+ * y_host [T, d], all enqueued on `stream`. Host buffers should be pinned
+ * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous; the
+ * caller synchronises the stream before reading y_host. Weights stay in
+ * device memory. Needs moe_workspace_size_host() bytes of workspace.
+ */
+MOE_API moe_status moe_workspace_size_host(const moe_cfg* cfg, int64_t T, size_t* bytes);
+MOE_API moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
+                            const float* b, const void* W1, const void* W3, const void* W2,
+                            const void* Ws1, const void* Ws3, const void* Ws2, void* y_host,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Reads (and optionally clears) the device-status word of a workspace used
+ * for T tokens with cfg: synchronises `stream`, writes the MOE_DEV_* bits
+ * to *bits, and returns MOE_ERR_DEVICE when any bit is set.
+ */
+MOE_API moe_status moe_device_status(const moe_cfg* cfg, int64_t T, void* ws, size_t ws_bytes, int clear,
+                             uint32_t* bits, void* stream);
+
+/*
+ * Stage timing hook for profilers and benchmarks. With n == 7, every later
+ * moe_forward / moe_forward_host call on this host thread records
+ * events[0..6] (cudaEvent_t handles owned by the caller, created on the
+ * stream's device) on its stream at the stage boundaries: before the
+ * router, after the router, after dispatch, after the row gather, after
+ * the SwiGLU GEMM, after the gate GEMM and after the combine. n == 0
+ * detaches. Any other n returns MOE_ERR_INVALID_ARG.
+ */
+MOE_API moe_status moe_set_stage_events(void* const* events, int32_t n);
+
+/* Human-readable name of a status code (static storage). */
+MOE_API const char* moe_status_string(moe_status status);
+
+/* cudaError_t value of the last MOE_ERR_CUDA on this host thread (0 if none). */
+MOE_API int32_t moe_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,242 @@
+// Dispatch: expert histogram, exclusive scan, expert-contiguous permutation
+// and the row gather that feeds the grouped GEMMs. This replaces the quoted
+// MoE.forward's bincount(...).tolist() and per-expert torch.where loop
+// ("DeepSeek-V3.2-Exp · Mixture of experts", quoted forward excerpt) with
+// three small kernels and no host round trip.
+//
+// Bit-exact by construction: a warp owns 32 consecutive tokens; for each
+// expert it forms a ballot of the tokens that chose it, so a pair's rank
+// inside the chunk is the popcount of the lower lanes, and chunk bases come
+// from a scan in (expert, chunk) order. No atomics decide any position.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kWarpsPerCta = 8;
+constexpr int kMaxWords = kMaxRouted / 32;
+
+struct ChunkArgs {
+  const int32_t* idx;
+  int64_t T;
+  int N, k;
+  int32_t* chunk_counts;     // [n_chunks, N]
+  const int32_t* chunk_base; // [n_chunks, N] (scatter pass)
+  const float* gates;        // [T, k]       (scatter pass)
+  int32_t* perm;
+  int32_t* slot_pos;
+  float* gate_perm;
+  unsigned* status;
+};
+
+// Pass 0 (counting) or 1 (scatter) over chunks of 32 tokens, one warp each.
+template <bool kScatter>
+__global__ void __launch_bounds__(32 * kWarpsPerCta) chunk_kernel(ChunkArgs a) {
+  __shared__ uint32_t bits[kWarpsPerCta][kMaxWords][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t c = (int64_t)blockIdx.x * kWarpsPerCta + w;
+  const int64_t n_chunks = (a.T + 31) / 32;
+  if (c >= n_chunks) return;
+  const int64_t t = c * 32 + lane;
+  const int W = (a.N + 31) / 32;
+  for (int i = 0; i < W; ++i) bits[w][i][lane] = 0u;
+  __syncwarp();
+  int32_t my[kMaxTopK];
+  if (t < a.T) {
+    for (int s = 0; s < a.k; ++s) {
+      int32_t e = a.idx[t * a.k + s];
+      my[s] = e;
+      if (e < 0 || e >= a.N) {
+        if (!kScatter) set_status(a.status, MOE_DEV_BAD_EXPERT);
+        my[s] = -1;
+        continue;
+      }
+      uint32_t m = 1u << (e & 31);
+      if (bits[w][e >> 5][lane] & m) {
+        if (!kScatter) set_status(a.status, MOE_DEV_DUP_EXPERT);
+        my[s] = -1;
+      }
+      bits[w][e >> 5][lane] |= m;
+    }
+  }
+  __syncwarp();
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int i = 0; i < W; ++i) {
+    const uint32_t word = bits[w][i][lane];
+    int my_count = 0;
+    for (int b = 0; b < 32; ++b) {
+      const bool has = (word >> b) & 1u;
+      const uint32_t m = __ballot_sync(0xffffffffu, has);
+      if (!kScatter) {
+        if (lane == b) my_count = __popc(m);
+      } else if (has) {
+        const int e = 32 * i + b;
+        const int32_t pos = a.chunk_base[c * a.N + e] + __popc(m & lt);
+        int slot = 0;
+        for (int s = 0; s < a.k; ++s)
+          if (my[s] == e) slot = s;
+        const int32_t flat = (int32_t)(t * a.k + slot);
+        a.perm[pos] = flat;
+        a.slot_pos[flat] = pos;
+        if (a.gates) a.gate_perm[pos] = a.gates[flat];
+      }
+    }
+    if (!kScatter) {
+      const int e = 32 * i + lane;
+      if (e < a.N) a.chunk_counts[c * a.N + e] = my_count;
+    }
+  }
+}
+
+// Exclusive scan of v over the whole block (blockDim.x a multiple of 32,
+// at most 1024); returns the prefix and writes the block total to *total.
+MOE_DEV int block_exclusive_scan(int v, int* total) {
+  __shared__ int warp_base[32];
+  __shared__ int block_total;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_base[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int x = lane < nw ? warp_base[lane] : 0;
+    int xi = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      int o = __shfl_up_sync(0xffffffffu, xi, off);
+      if (lane >= off) xi += o;
+    }
+    if (lane < nw) warp_base[lane] = xi - x;
+    if (lane == 31) block_total = xi;
+  }
+  __syncthreads();
+  const int res = warp_base[w] + incl - v;
+  *total = block_total;
+  __syncthreads();  // the shared slots are reused by the next call
+  return res;
+}
+
+struct ScanArgs {
+  int32_t* chunk_counts;  // in: counts per chunk; out (as chunk_base): absolute positions
+  int64_t n_chunks, T;
+  int N, ns, F, nsF, d;
+  int bm, bn1, bn2;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* grp_row0;
+  int32_t* grp_rows;
+  int32_t* unit_base1;
+  int32_t* unit_base2;
+};
+
+// One CTA of 1024 threads: per-expert totals and chunk bases, offsets, and the
+// GEMM unit tables (groups 0..N-1 routed, group N the shared MLP).
+__global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a, int32_t* chunk_base) {
+  const int tid = threadIdx.x;
+  int cnt = 0;
+  if (tid < a.N) {
+    int run = 0;
+    for (int64_t c = 0; c < a.n_chunks; ++c) {
+      int v = a.chunk_counts[c * a.N + tid];
+      chunk_base[c * a.N + tid] = run;
+      run += v;
+    }
+    cnt = run;
+  }
+  int total;
+  const int off = block_exclusive_scan(cnt, &total);
+  if (tid < a.N) {
+    a.counts[tid] = cnt;
+    a.offsets[tid] = off;
+    for (int64_t c = 0; c < a.n_chunks; ++c) chunk_base[c * a.N + tid] += off;
+  }
+  if (tid == 0) a.offsets[a.N] = total;
+
+  // unit tables over groups g = 0..N (N = shared MLP)
+  int rows = 0, row0 = 0, u1 = 0, u2 = 0;
+  if (tid < a.N) {
+    rows = cnt;
+    row0 = off;
+  } else if (tid == a.N && a.ns > 0) {
+    rows = (int)a.T;
+    row0 = 0;
+  }
+  if (tid <= a.N) {
+    const int mt = (rows + a.bm - 1) / a.bm;
+    const int cols1 = tid < a.N ? a.F : a.nsF;
+    u1 = mt * ((cols1 + a.bn1 - 1) / a.bn1);
+    u2 = mt * ((a.d + a.bn2 - 1) / a.bn2);
+    a.grp_rows[tid] = rows;
+    a.grp_row0[tid] = row0;
+  }
+  int tot1, tot2;
+  const int b1 = block_exclusive_scan(u1, &tot1);
+  const int b2 = block_exclusive_scan(u2, &tot2);
+  if (tid <= a.N) {
+    a.unit_base1[tid] = b1;
+    a.unit_base2[tid] = b2;
+  }
+  if (tid == 0) {
+    a.unit_base1[a.N + 1] = tot1;
+    a.unit_base2[a.N + 1] = tot2;
+  }
+}
+
+template <typename TV>
+__global__ void __launch_bounds__(256) gather_kernel(const TV* __restrict__ x,
+                                                     const int32_t* __restrict__ perm,
+                                                     const int32_t* __restrict__ n_rows, int64_t R,
+                                                     int k, int vecs, TV* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = *n_rows;  // pairs actually placed (== R unless the indices were invalid)
+  if (rows < R) R = rows < 0 ? 0 : rows;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += warps) {
+    const int64_t t = perm[r] / k;
+    const TV* src = x + t * vecs;
+    TV* dst = x_perm + r * vecs;
+    for (int v = lane; v < vecs; v += 32) dst[v] = src[v];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const Problem& p, const DispatchBuffers& db, int bm, int bn1, int bn2,
+                            cudaStream_t s) {
+  const int64_t n_chunks = (p.T + 31) / 32;
+  const unsigned blocks = (unsigned)((n_chunks + kWarpsPerCta - 1) / kWarpsPerCta);
+  ChunkArgs ca{db.idx, p.T, p.N, p.k, db.chunk_counts, db.chunk_base, db.gates, db.perm,
+               db.slot_pos, db.gate_perm, db.status};
+  cudaError_t err = cudaMemsetAsync(db.slot_pos, 0xFF, (size_t)p.R * sizeof(int32_t), s);
+  if (err != cudaSuccess) return err;
+  chunk_kernel<false><<<blocks, 32 * kWarpsPerCta, 0, s>>>(ca);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  ScanArgs sa{db.chunk_counts, n_chunks, p.T, p.N, p.ns, p.F, p.nsF, p.d, bm, bn1, bn2,
+              db.counts, db.offsets, db.grp_row0, db.grp_rows, db.unit_base1, db.unit_base2};
+  scan_kernel<<<1, 1024, 0, s>>>(sa, db.chunk_base);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  chunk_kernel<true><<<blocks, 32 * kWarpsPerCta, 0, s>>>(ca);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm,
+                          const int32_t* n_rows, void* x_perm, cudaStream_t s) {
+  if (p.R == 0) return cudaSuccess;
+  const int vecs = (int)((int64_t)p.d * p.elem / 16);
+  int64_t want = (p.R + 7) / 8;
+  int64_t cap = (int64_t)device_sm_count() * 16;
+  unsigned blocks = (unsigned)(want < cap ? want : cap);
+  gather_kernel<uint4><<<blocks, 256, 0, s>>>((const uint4*)x, perm, n_rows, p.R, p.k, vecs,
+                                              (uint4*)x_perm);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,387 @@
+// C ABI of the layer (declared in include/moe_b200.h): argument checks,
+// workspace carving and the launch sequence
+//   router -> dispatch -> gather -> SwiGLU GEMM -> gate GEMM -> combine,
+// all on the caller's stream with no host synchronisation.
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+thread_local int32_t g_last_cuda_error = 0;
+constexpr int kStageEvents = 7;
+thread_local cudaEvent_t g_stage_events[kStageEvents] = {};
+thread_local bool g_stage_events_on = false;
+
+cudaError_t mark_stage(int i, cudaStream_t s) {
+  return g_stage_events_on ? cudaEventRecord(g_stage_events[i], s) : cudaSuccess;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int32_t)e;
+  return MOE_ERR_CUDA;
+}
+}  // namespace
+
+int device_sm_count() {
+  static int cached_dev = -1, cached_sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cached_sms;
+  if (dev != cached_dev) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0) {
+      cached_sms = sms;
+      cached_dev = dev;
+    }
+  }
+  return cached_sms;
+}
+
+moe_status make_problem(const moe_cfg* cfg, int64_t T, Problem* p) {
+  if (!cfg || !p || T < 0) return MOE_ERR_INVALID_ARG;
+  const moe_cfg& c = *cfg;
+  if (c.d <= 0 || c.d_ff <= 0 || c.n_routed <= 0 || c.n_shared < 0 || c.top_k <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c.d % 8 || c.d_ff % 8) return MOE_ERR_INVALID_ARG;
+  if (c.top_k > c.n_routed) return MOE_ERR_INVALID_ARG;
+  const int G = c.n_groups <= 0 ? 1 : c.n_groups;
+  const int TG = G == 1 ? 1 : c.topk_groups;
+  if (c.n_routed % G || TG < 1 || TG > G) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)c.top_k > (int64_t)TG * (c.n_routed / G)) return MOE_ERR_INVALID_ARG;
+  if (c.score_fn != MOE_SOFTMAX && c.score_fn != MOE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (c.group_score != MOE_GROUP_TOP2_SUM && c.group_score != MOE_GROUP_MAX) return MOE_ERR_INVALID_ARG;
+  if (G > 1 && c.group_score == MOE_GROUP_TOP2_SUM && c.n_routed / G < 2) return MOE_ERR_INVALID_ARG;
+  if (c.dtype != MOE_F32 && c.dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (!(c.route_scale == c.route_scale)) return MOE_ERR_INVALID_ARG;  // NaN
+  // implemented range
+  if (c.n_routed > kMaxRouted || c.top_k > kMaxTopK || G > 32) return MOE_ERR_UNSUPPORTED;
+  const int64_t nsF64 = (int64_t)c.n_shared * c.d_ff;
+  if (nsF64 > (1 << 30) || (int64_t)c.n_routed * c.d_ff > (1ll << 31) ||
+      (int64_t)c.n_routed * c.d > (1ll << 31))
+    return MOE_ERR_UNSUPPORTED;
+  if (T * (int64_t)c.top_k + T > (1ll << 31) - 1) return MOE_ERR_UNSUPPORTED;
+  p->T = T;
+  p->d = c.d;
+  p->F = c.d_ff;
+  p->N = c.n_routed;
+  p->ns = c.n_shared;
+  p->k = c.top_k;
+  p->G = G;
+  p->TG = TG;
+  p->score_fn = c.score_fn;
+  p->normalize = c.normalize != 0;
+  p->group_score = c.group_score;
+  p->dtype = c.dtype;
+  p->route_scale = c.route_scale;
+  p->R = T * c.top_k;
+  p->nsF = (int)nsF64;
+  p->elem = c.dtype == MOE_BF16 ? 2 : 4;
+  return MOE_OK;
+}
+
+Layout make_layout(const Problem& p) {
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  const int64_t T = p.T, N = p.N, R = p.R;
+  L.n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
+  L.status = take(256);
+  L.logits = take((size_t)T * N * 4);
+  L.idx = take((size_t)R * 4);
+  L.gates = take((size_t)R * 4);
+  L.chunk_counts = take((size_t)L.n_chunks * N * 4);
+  L.chunk_base = take((size_t)L.n_chunks * N * 4);
+  L.counts = take((size_t)N * 4);
+  L.offsets = take((size_t)(N + 1) * 4);
+  L.grp_row0 = take((size_t)(N + 1) * 4);
+  L.grp_rows = take((size_t)(N + 1) * 4);
+  L.unit_base1 = take((size_t)(N + 2) * 4);
+  L.unit_base2 = take((size_t)(N + 2) * 4);
+  L.perm = take((size_t)R * 4);
+  L.slot_pos = take((size_t)R * 4);
+  L.gate_perm = take((size_t)R * 4);
+  L.x_perm = take((size_t)R * p.d * p.elem);
+  L.h_perm = take((size_t)R * p.F * p.elem);
+  L.h_sh = take((size_t)T * p.nsF * p.elem);
+  L.y_rows = take((size_t)(R + T) * p.d * p.elem);
+  L.total = off;
+  L.x_stage = take((size_t)T * p.d * p.elem);
+  L.y_stage = take((size_t)T * p.d * p.elem);
+  L.total_host = off;
+  return L;
+}
+
+namespace {
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status check_ws(const Layout& L, void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
+  (void)L;
+  return MOE_OK;
+}
+
+moe_status run_router(const Problem& p, const Layout& L, const void* x, const void* W_r,
+                      const float* b, int32_t* idx, float* gates, void* ws, cudaStream_t s) {
+  cudaError_t e = launch_router(p, x, W_r, b, at<float>(ws, L.logits), idx, gates, s);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+DispatchBuffers dispatch_buffers(const Layout& L, void* ws, const int32_t* idx, const float* gates) {
+  DispatchBuffers db;
+  db.idx = idx;
+  db.chunk_counts = at<int32_t>(ws, L.chunk_counts);
+  db.chunk_base = at<int32_t>(ws, L.chunk_base);
+  db.counts = at<int32_t>(ws, L.counts);
+  db.offsets = at<int32_t>(ws, L.offsets);
+  db.grp_row0 = at<int32_t>(ws, L.grp_row0);
+  db.grp_rows = at<int32_t>(ws, L.grp_rows);
+  db.unit_base1 = at<int32_t>(ws, L.unit_base1);
+  db.unit_base2 = at<int32_t>(ws, L.unit_base2);
+  db.perm = at<int32_t>(ws, L.perm);
+  db.slot_pos = at<int32_t>(ws, L.slot_pos);
+  db.gate_perm = at<float>(ws, L.gate_perm);
+  db.gates = gates;
+  db.status = at<unsigned>(ws, L.status);
+  return db;
+}
+
+moe_status forward_device(const Problem& p, const Layout& L, const void* x, const void* W_r,
+                          const float* b, const void* W1, const void* W3, const void* W2,
+                          const void* Ws1, const void* Ws3, const void* Ws2, void* y,
+                          int32_t* idx_out, float* gates_out, void* ws, cudaStream_t s) {
+  int32_t* idx = at<int32_t>(ws, L.idx);
+  float* gates = at<float>(ws, L.gates);
+  cudaError_t e0 = cudaMemsetAsync(at<void>(ws, L.status), 0, 4, s);
+  if (e0 == cudaSuccess) e0 = mark_stage(0, s);
+  if (e0 != cudaSuccess) return cuda_fail(e0);
+  moe_status st = run_router(p, L, x, W_r, b, idx, gates, ws, s);
+  if (st != MOE_OK) return st;
+  if ((e0 = mark_stage(1, s)) != cudaSuccess) return cuda_fail(e0);
+  const bool tc = p.dtype == MOE_BF16;
+  DispatchBuffers db = dispatch_buffers(L, ws, idx, gates);
+  cudaError_t e = launch_dispatch(p, db, tc ? kTcBM : kSimtBM, tc ? kTcBN1 : kSimtBN,
+                                  tc ? kTcBN2 : kSimtBN, s);
+  if (e == cudaSuccess) e = mark_stage(2, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = launch_gather(p, x, db.perm, db.offsets + p.N, at<void>(ws, L.x_perm), s);
+  if (e == cudaSuccess) e = mark_stage(3, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  GemmArgs ga;
+  ga.x = x;
+  ga.x_perm = at<void>(ws, L.x_perm);
+  ga.W1 = W1;
+  ga.W3 = W3;
+  ga.W2 = W2;
+  ga.Ws1 = p.ns ? Ws1 : nullptr;
+  ga.Ws3 = p.ns ? Ws3 : nullptr;
+  ga.Ws2 = p.ns ? Ws2 : nullptr;
+  ga.h_perm = at<void>(ws, L.h_perm);
+  ga.h_sh = at<void>(ws, L.h_sh);
+  ga.y_rows = at<void>(ws, L.y_rows);
+  ga.grp_row0 = db.grp_row0;
+  ga.grp_rows = db.grp_rows;
+  ga.unit_base1 = db.unit_base1;
+  ga.unit_base2 = db.unit_base2;
+  ga.gate_perm = db.gate_perm;
+  ga.status = db.status;
+  e = tc ? launch_expert_gemms_tc(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr)
+         : launch_expert_gemms_simt(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr);
+  if (e == cudaSuccess) e = mark_stage(5, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = launch_combine(p, ga.y_rows, db.slot_pos, idx, y, s);
+  if (e == cudaSuccess) e = mark_stage(6, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (idx_out) {
+    e = cudaMemcpyAsync(idx_out, idx, (size_t)p.R * 4, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (gates_out) {
+    e = cudaMemcpyAsync(gates_out, gates, (size_t)p.R * 4, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return MOE_OK;
+}
+
+moe_status check_weights(const Problem& p, const void* W_r, const float* b, const void* W1,
+                         const void* W3, const void* W2, const void* Ws1, const void* Ws3,
+                         const void* Ws2) {
+  if (!W_r || !W1 || !W3 || !W2) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(W_r) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2)) return MOE_ERR_INVALID_ARG;
+  if (b && (reinterpret_cast<uintptr_t>(b) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (p.ns > 0) {
+    if (!Ws1 || !Ws3 || !Ws2) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(Ws1) || !aligned16(Ws3) || !aligned16(Ws2)) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_workspace_size(const moe_cfg* cfg, int64_t T, size_t* bytes) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = make_layout(p).total;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_size_host(const moe_cfg* cfg, int64_t T, size_t* bytes) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = make_layout(p).total_host;
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_cfg* cfg, int64_t T, const void* x, const void* W_r, const float* b,
+                     int32_t* topk_idx, float* gates, void* ws, size_t ws_bytes, void* stream) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !W_r || !topk_idx || !gates || !aligned16(x) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
+  Layout L = make_layout(p);
+  if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
+  return run_router(p, L, x, W_r, b, topk_idx, gates, ws, (cudaStream_t)stream);
+}
+
+moe_status moe_dispatch(const moe_cfg* cfg, int64_t T, const int32_t* topk_idx, int32_t* counts,
+                        int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!topk_idx) return MOE_ERR_INVALID_ARG;
+  Layout L = make_layout(p);
+  if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  DispatchBuffers db = dispatch_buffers(L, ws, topk_idx, nullptr);
+  const bool tc = p.dtype == MOE_BF16;
+  cudaError_t e = cudaMemsetAsync(db.status, 0, 4, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = launch_dispatch(p, db, tc ? kTcBM : kSimtBM, tc ? kTcBN1 : kSimtBN,
+                                  tc ? kTcBN2 : kSimtBN, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (counts && (e = cudaMemcpyAsync(counts, db.counts, (size_t)p.N * 4, cudaMemcpyDeviceToDevice, s)))
+    return cuda_fail(e);
+  if (offsets &&
+      (e = cudaMemcpyAsync(offsets, db.offsets, (size_t)(p.N + 1) * 4, cudaMemcpyDeviceToDevice, s)))
+    return cuda_fail(e);
+  if (perm && (e = cudaMemcpyAsync(perm, db.perm, (size_t)p.R * 4, cudaMemcpyDeviceToDevice, s)))
+    return cuda_fail(e);
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_cfg* cfg, int64_t T, const void* x, const void* W_r, const float* b,
+                       const void* W1, const void* W3, const void* W2, const void* Ws1,
+                       const void* Ws3, const void* Ws2, void* y, int32_t* topk_idx_out,
+                       float* gates_out, void* ws, size_t ws_bytes, void* stream) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_weights(p, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2)) != MOE_OK) return st;
+  Layout L = make_layout(p);
+  if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
+  return forward_device(p, L, x, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y, topk_idx_out, gates_out, ws,
+                        (cudaStream_t)stream);
+}
+
+moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
+                            const float* b, const void* W1, const void* W3, const void* W2,
+                            const void* Ws1, const void* Ws3, const void* Ws2, void* y_host,
+                            void* ws, size_t ws_bytes, void* stream) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
+  if ((st = check_weights(p, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2)) != MOE_OK) return st;
+  Layout L = make_layout(p);
+  if ((st = check_ws(L, ws, ws_bytes, L.total_host)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t bytes = (size_t)p.T * p.d * p.elem;
+  void* xd = at<void>(ws, L.x_stage);
+  void* yd = at<void>(ws, L.y_stage);
+  cudaError_t e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  st = forward_device(p, L, xd, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, yd, nullptr, nullptr, ws, s);
+  if (st != MOE_OK) return st;
+  e = cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return MOE_OK;
+}
+
+moe_status moe_device_status(const moe_cfg* cfg, int64_t T, void* ws, size_t ws_bytes, int clear,
+                             uint32_t* bits, void* stream) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
+  if (st != MOE_OK) return st;
+  if (!bits) return MOE_ERR_INVALID_ARG;
+  Layout L = make_layout(p);
+  if ((st = check_ws(L, ws, ws_bytes, 256)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, at<void>(ws, L.status), 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (clear) {
+    e = cudaMemsetAsync(at<void>(ws, L.status), 0, 4, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  *bits = host;
+  return host ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+const char* moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int32_t moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+moe_status moe_set_stage_events(void* const* events, int32_t n) {
+  if (n == 0) {
+    g_stage_events_on = false;
+    return MOE_OK;
+  }
+  if (n != kStageEvents || !events) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < kStageEvents; ++i) {
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+    g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  g_stage_events_on = true;
+  return MOE_OK;
+}
+
+}  // extern "C"

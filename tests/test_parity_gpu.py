@@ -1,0 +1,207 @@
+"""GPU parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+Small layers (full oracle, several tiles and ragged tails) and the five
+layer configurations at full size (oracle on sampled tokens; routing on all
+tokens). Inputs come from the seeded generator on both sides."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+from moe_inputs import device as mdev
+import mixture_experts_layer_group_b200 as moe
+
+from gpu_helpers import (TOL, cfg_of, check_routing, f64, host_expert_fn, host_shared64, oracle_forward,
+                         rel_fro, router_cfg_of, run_forward, t2np64, workspace)
+
+pytestmark = pytest.mark.gpu
+
+LS = mi.LayerShape
+# small layers whose oracle runs in seconds; each spans several tiles and has ragged tails
+SMALL = {
+    "v3_like_small": LS("v3_like_small", T=300, d=512, n_routed=32, n_shared=1, d_ff=256, top_k=4,
+                        score="sigmoid", n_groups=4, topk_groups=2, normalize=True, route_scale=2.5, seed=11,
+                        bias=True),
+    "softmax_ragged": LS("softmax_ragged", T=517, d=384, n_routed=20, n_shared=2, d_ff=384, top_k=3,
+                         score="softmax", seed=12),
+    "group_max_odd": LS("group_max_odd", T=129, d=256, n_routed=63, n_shared=0, d_ff=128, top_k=6,
+                        score="sigmoid", n_groups=9, topk_groups=3, normalize=True, route_scale=1.0,
+                        group_score="max", seed=13, bias=True),
+    "single_token": LS("single_token", T=1, d=512, n_routed=16, n_shared=1, d_ff=256, top_k=2,
+                       score="softmax", seed=14),
+    "tiny_f32": LS("tiny_f32", T=77, d=136, n_routed=12, n_shared=1, d_ff=200, top_k=3, score="sigmoid",
+                   normalize=True, route_scale=2.5, dtype="f32", seed=15, bias=True),
+    "gshard_tiny_f32": mi.SHAPES["gshard_tiny_f32"],
+}
+
+
+@pytest.fixture(autouse=True)
+def _lib():
+    from mixture_experts_layer_group_b200 import build
+    from moe_inputs import build as gb
+    build.build()
+    gb.build_device()
+    torch.cuda.set_device(0)
+    yield
+    torch.cuda.empty_cache()
+
+
+def full_oracle_check(s, w=None, x=None):
+    w = mdev.device_all(s) if w is None else w
+    x = mdev.device_tensor(s, "x") if x is None else x
+    y, gidx, ggates = run_forward(s, w, x)
+    h = mi.host_all(s)
+    x64 = f64(h["x"])
+    W_r64 = f64(h["W_r"])
+    b = None if h["b"] is None else h["b"].astype(np.float64)
+    expert = lambda e: (f64(h["W1"][e]), f64(h["W3"][e]), f64(h["W2"][e]))  # noqa: E731
+    shared = None if s.n_shared == 0 else (f64(h["Ws1"]), f64(h["Ws3"]), f64(h["Ws2"]))
+    ref, r = oracle_forward(s, x64, W_r64, b, expert, shared, gidx)
+    n_flag, n_diff = check_routing(gidx, ggates, r, router_cfg_of(s))
+    err = rel_fro(t2np64(y), ref)
+    assert err <= TOL[s.dtype], (s.name, err)
+    return err, gidx, y
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_layer_full_parity(name):
+    full_oracle_check(SMALL[name])
+
+
+def test_dispatch_bit_exact_and_edge_cases():
+    s = SMALL["v3_like_small"]
+    cfg = cfg_of(s)
+    for T, idx in [(300, None), (1, None), (33, None), (257, "hot"), (64, "reverse")]:
+        if idx is None:
+            x = mdev.device_tensor(s.with_(T=T), "x")
+            w = mdev.device_all(s)
+            ws = workspace(cfg, T)
+            gi = torch.empty((T, s.top_k), dtype=torch.int32, device="cuda")
+            gg = torch.empty((T, s.top_k), dtype=torch.float32, device="cuda")
+            moe.route(cfg, T, x, w["W_r"], w["b"], gi, gg, ws)
+            torch.cuda.synchronize()
+            idx_np = gi.cpu().numpy()
+        elif idx == "hot":  # every token picks the same experts
+            idx_np = np.tile(np.array([[5, 2, 31, 0]], dtype=np.int32), (T, 1))
+        else:  # experts in descending order per token
+            idx_np = np.stack([np.random.default_rng(t).choice(32, 4, replace=False) for t in range(T)])
+            idx_np = -np.sort(-idx_np, axis=1).astype(np.int32)
+        ws = workspace(cfg, T)
+        counts = torch.empty(s.n_routed, dtype=torch.int32, device="cuda")
+        offsets = torch.empty(s.n_routed + 1, dtype=torch.int32, device="cuda")
+        perm = torch.empty(T * s.top_k, dtype=torch.int32, device="cuda")
+        moe.dispatch(cfg, T, torch.from_numpy(idx_np).cuda(), counts, offsets, perm, ws)
+        torch.cuda.synchronize()
+        assert moe.device_status(cfg, T, ws) == 0
+        c_ref, o_ref, p_ref = oracle.permutation(idx_np.astype(np.int64), s.n_routed)
+        assert (counts.cpu().numpy() == c_ref).all()
+        assert (offsets.cpu().numpy() == o_ref).all()
+        assert (perm.cpu().numpy() == p_ref).all()
+
+
+def test_dispatch_flags_invalid_indices():
+    s = SMALL["v3_like_small"]
+    cfg = cfg_of(s)
+    T = 40
+    idx = torch.zeros((T, s.top_k), dtype=torch.int32)
+    idx[:] = torch.tensor([1, 2, 3, 4], dtype=torch.int32)
+    idx[7, 2] = 99       # out of range
+    idx[9, 3] = 1        # duplicate of slot 0
+    ws = workspace(cfg, T)
+    moe.dispatch(cfg, T, idx.cuda(), None, None, None, ws)
+    torch.cuda.synchronize()
+    bits = moe.device_status(cfg, T, ws)
+    assert bits & moe.MOE_DEV_BAD_EXPERT and bits & moe.MOE_DEV_DUP_EXPERT
+
+
+def test_route_matches_forward_routing_and_is_deterministic():
+    s = SMALL["v3_like_small"]
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    y1, i1, g1 = run_forward(s, w, x)
+    y2, i2, g2 = run_forward(s, w, x)
+    assert torch.equal(y1, y2) and (i1 == i2).all() and (g1 == g2).all()
+    cfg = cfg_of(s)
+    ws = workspace(cfg, s.T)
+    gi = torch.empty((s.T, s.top_k), dtype=torch.int32, device="cuda")
+    gg = torch.empty((s.T, s.top_k), dtype=torch.float32, device="cuda")
+    moe.route(cfg, s.T, x, w["W_r"], w["b"], gi, gg, ws)
+    torch.cuda.synchronize()
+    assert (gi.cpu().numpy() == i1).all() and (gg.cpu().numpy() == g1).all()
+
+
+def test_identical_experts_invariant():
+    # every routed expert identical, normalised gates: y = 2.5 FFN(x) + shared(x) whatever the routing
+    s = SMALL["v3_like_small"]
+    w = mdev.device_all(s)
+    for nm in ("W1", "W3", "W2"):
+        w[nm] = w[nm][:1].expand_as(w[nm]).contiguous()
+    x = mdev.device_tensor(s, "x")
+    y, gidx, _ = run_forward(s, w, x)
+    h = mi.host_all(s)
+    x64 = f64(h["x"])
+    e0 = (f64(h["W1"][0]), f64(h["W3"][0]), f64(h["W2"][0]))
+    ref = 2.5 * oracle.expert_ffn(x64, *e0) + oracle.expert_ffn(x64, f64(h["Ws1"]), f64(h["Ws3"]), f64(h["Ws2"]))
+    assert rel_fro(t2np64(y), ref) <= TOL["bf16"]
+
+
+def test_forward_host_matches_device_forward():
+    s = SMALL["softmax_ragged"]
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    y_dev, _, _ = run_forward(s, w, x)
+    cfg = cfg_of(s)
+    ws = workspace(cfg, s.T, host=True)
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    moe.forward_host(cfg, s.T, xh, w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"],
+                     yh, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y_dev.cpu())
+
+
+def test_abi_errors_on_device_buffers():
+    s = SMALL["v3_like_small"]
+    cfg = cfg_of(s)
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    y = torch.empty_like(x)
+    small = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(moe.MoeError) as ei:
+        moe.forward(cfg, s.T, x, w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"], y,
+                    small)
+    assert ei.value.status == 3
+    ws = workspace(cfg, s.T)
+    with pytest.raises(moe.MoeError):
+        moe.forward(cfg, s.T, x, w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], None, None, None, y, ws)
+    moe.forward(cfg, 0, x, w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"], y, ws)
+
+
+# ------------------------------------------------------------- full size ----
+
+SAMPLES = {"gshard_tiny_f32": None, "dsmoe_2b_bf16": 64, "v2_layer_bf16": 16, "v3_prefill_bf16": 16,
+           "v3_decode_bf16": None}
+
+
+@pytest.mark.parametrize("name", mi.ORDER)
+def test_full_size_config(name):
+    s = mi.SHAPES[name]
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    y, gidx, ggates = run_forward(s, w, x)
+    del w
+    torch.cuda.empty_cache()
+    # routing of every token
+    x64 = f64(mi.host_tensor(s, "x").reshape(s.T, s.d))
+    W_r64 = f64(mi.host_tensor(s, "W_r").reshape(s.n_routed, s.d))
+    b = mi.host_tensor(s, "b").astype(np.float64) if s.bias else None
+    rcfg = router_cfg_of(s)
+    r = oracle.route(x64, W_r64, b, rcfg)
+    check_routing(gidx, ggates, r, rcfg)
+    # outputs on sampled tokens (all tokens for the small ones)
+    n = SAMPLES[name]
+    rows = np.arange(s.T) if n is None else np.sort(np.random.default_rng(s.seed).choice(s.T, n, replace=False))
+    ref, _ = oracle_forward(s, x64[rows], W_r64, b, host_expert_fn(s), host_shared64(s), gidx[rows])
+    err = rel_fro(t2np64(y[torch.from_numpy(rows).cuda()]), ref)
+    assert err <= TOL[s.dtype], (name, err)
