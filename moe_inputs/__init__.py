@@ -87,6 +87,11 @@ SHAPES = {
                                  d_ff=2048, top_k=8, score="sigmoid", n_groups=8, topk_groups=4,
                                  normalize=True, route_scale=2.5, seed=4, bias=True, zipf_s=1.2),
 }
+# A V3-shaped layer cut to 32 routed experts (2.9 GB of weights, still far
+# beyond L2) for full-metric profiler captures of the same kernels.
+SHAPES["v3_profile_32e"] = LayerShape("v3_profile_32e", T=1024, d=7168, n_routed=32, n_shared=1, d_ff=2048,
+                                      top_k=8, score="sigmoid", n_groups=8, topk_groups=4, normalize=True,
+                                      route_scale=2.5, seed=5, bias=True)
 ORDER = ["gshard_tiny_f32", "dsmoe_2b_bf16", "v2_layer_bf16", "v3_prefill_bf16", "v3_decode_bf16"]
 
 
