@@ -197,6 +197,32 @@ MOE_API moe_status moe_device_status(const moe_cfg* cfg, int64_t T, void* ws, si
  */
 MOE_API moe_status moe_set_stage_events(void* const* events, int32_t n);
 
+/*
+ * Router that allocates nothing and takes no workspace. The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate
+ * device memory for scratch -- a plugin whose host framework owns all device
+ * memory and passes it no workspace, or a serving loop with a fixed memory
+ * budget that must not call cudaMalloc (which can synchronise the device)
+ * once it runs.
+ *   Same arguments, outputs and results as moe_route, without ws/ws_bytes.
+ *   Scratch: the fp32 logits (T * n_routed * 4 bytes) go to a fixed 8 MiB
+ *     array inside the library, reserved on every GPU that loads the
+ *     library until the process exits. T * n_routed * 4 > 8 MiB (for
+ *     example T > 8192 at n_routed = 256) returns MOE_ERR_UNSUPPORTED; use
+ *     moe_route with a workspace for those sizes.
+ *   Set-up: the first call on a device (with that device current) looks up
+ *     the array's device address and caches it; make that first call before
+ *     any stream capture. It never calls cudaMalloc, cudaFree or any other
+ *     allocating routine.
+ *   Sharing: every call on a device uses the same array and leaves the last
+ *     call's logits in it (each call overwrites every value it reads, so
+ *     nothing needs clearing). Calls whose work overlaps on the GPU -- on
+ *     different streams, or from different host threads -- race on the
+ *     array and may return wrong routing: serialise them, e.g. on one stream.
+ */
+MOE_API moe_status moe_route_noalloc(const moe_cfg* cfg, int64_t T, const void* x, const void* W_r,
+                                     const float* b, int32_t* topk_idx, float* gates, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 MOE_API const char* moe_status_string(moe_status status);
 

@@ -107,4 +107,7 @@ cudaError_t launch_combine(const Problem& p, const void* y_rows, const int32_t* 
 
 int device_sm_count();
 
+// Keeps e as this host thread's moe_last_cuda_error() value.
+void record_cuda_error(cudaError_t e);
+
 }  // namespace moe

@@ -29,6 +29,8 @@ moe_status cuda_fail(cudaError_t e) {
 }
 }  // namespace
 
+void record_cuda_error(cudaError_t e) { g_last_cuda_error = (int32_t)e; }
+
 int device_sm_count() {
   static int cached_dev = -1, cached_sms = 148;
   int dev = 0;
