@@ -48,44 +48,34 @@ struct Io<float> {
   }
 };
 
-// One CTA per token; each thread owns 16-byte column vectors.
-template <typename TE>
-__global__ void __launch_bounds__(128) combine_kernel(const uint4* __restrict__ y_rows,
-                                                      const int32_t* __restrict__ slot_pos,
-                                                      const int32_t* __restrict__ idx, int64_t T,
-                                                      int k, int N, int has_shared, int64_t R,
-                                                      int vecs, uint4* __restrict__ y) {
+// One CTA per token; each thread owns 16-byte column vectors. slot_pos
+// lists the token's rows in ascending expert order (written that way by the
+// dispatch), -1 for a pair that was never placed.
+template <typename TE, int KMAX>
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_rows,
+                                                      const int32_t* __restrict__ slot_pos, int64_t T,
+                                                      int k, int has_shared, int64_t R, int vecs,
+                                                      uint4* __restrict__ y) {
   constexpr int P = Io<TE>::kPerVec;
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    // slots sorted by ascending expert index (k <= 16, insertion sort)
-    int64_t rows[kMaxTopK + 1];
-    int experts[kMaxTopK];
-    int n = 0;
-    for (int s = 0; s < k; ++s) {
-      const int e = idx[t * k + s];
-      const int32_t pos = slot_pos[t * k + s];
-      if (e < 0 || e >= N || pos < 0 || pos >= R) continue;  // unplaced pair: contributes nothing
-      int j = n++;
-      while (j > 0 && experts[j - 1] > e) {
-        experts[j] = experts[j - 1];
-        rows[j] = rows[j - 1];
-        --j;
-      }
-      experts[j] = e;
-      rows[j] = pos;
+    int32_t rows[KMAX + 1];  // row indices < R + T < 2^31
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) {
+      const int32_t pos = s < k ? __ldg(slot_pos + t * k + s) : -1;
+      rows[s] = (pos >= 0 && pos < R) ? pos : -1;
     }
-    if (has_shared) rows[n++] = R + t;
+    rows[KMAX] = has_shared ? (int32_t)(R + t) : -1;
     for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
+      uint4 buf[KMAX + 1];
+#pragma unroll
+      for (int s = 0; s < KMAX + 1; ++s)
+        if (rows[s] >= 0) buf[s] = __ldg(y_rows + (int64_t)rows[s] * vecs + v);
       float acc[P];
 #pragma unroll
       for (int i = 0; i < P; ++i) acc[i] = 0.f;
-      uint4 buf[kMaxTopK + 1];
 #pragma unroll
-      for (int s = 0; s < kMaxTopK + 1; ++s)
-        if (s < n) buf[s] = y_rows[rows[s] * vecs + v];
-#pragma unroll
-      for (int s = 0; s < kMaxTopK + 1; ++s)
-        if (s < n) Io<TE>::add(buf[s], acc);
+      for (int s = 0; s < KMAX + 1; ++s)
+        if (rows[s] >= 0) Io<TE>::add(buf[s], acc);
       y[t * vecs + v] = Io<TE>::pack(acc);
     }
   }
@@ -93,17 +83,26 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint4* __restrict__ 
 
 }  // namespace
 
-cudaError_t launch_combine(const Problem& p, const void* y_rows, const int32_t* slot_pos,
-                           const int32_t* idx, void* y, cudaStream_t s) {
+cudaError_t launch_combine(const Problem& p, const void* y_rows, const int32_t* slot_pos, void* y,
+                           cudaStream_t s) {
   const int vecs = (int)((int64_t)p.d * p.elem / 16);
+  const int threads = vecs >= 256 ? 256 : (vecs >= 128 ? 128 : 64);
   int64_t cap = (int64_t)device_sm_count() * 16;
   unsigned blocks = (unsigned)(p.T < cap ? p.T : cap);
-  if (p.dtype == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<blocks, 128, 0, s>>>((const uint4*)y_rows, slot_pos, idx, p.T,
-                                                        p.k, p.N, p.ns > 0, p.R, vecs, (uint4*)y);
-  else
-    combine_kernel<float><<<blocks, 128, 0, s>>>((const uint4*)y_rows, slot_pos, idx, p.T, p.k,
-                                                p.N, p.ns > 0, p.R, vecs, (uint4*)y);
+  const uint4* yr = (const uint4*)y_rows;
+  const int sh = p.ns > 0;
+  if (p.dtype == MOE_BF16) {
+    if (p.k <= 8)
+      combine_kernel<__nv_bfloat16, 8><<<blocks, threads, 0, s>>>(yr, slot_pos, p.T, p.k, sh, p.R, vecs, (uint4*)y);
+    else
+      combine_kernel<__nv_bfloat16, kMaxTopK><<<blocks, threads, 0, s>>>(yr, slot_pos, p.T, p.k, sh, p.R, vecs,
+                                                                        (uint4*)y);
+  } else {
+    if (p.k <= 8)
+      combine_kernel<float, 8><<<blocks, threads, 0, s>>>(yr, slot_pos, p.T, p.k, sh, p.R, vecs, (uint4*)y);
+    else
+      combine_kernel<float, kMaxTopK><<<blocks, threads, 0, s>>>(yr, slot_pos, p.T, p.k, sh, p.R, vecs, (uint4*)y);
+  }
   return cudaGetLastError();
 }
 

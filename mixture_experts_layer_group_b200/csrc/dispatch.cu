@@ -15,7 +15,6 @@ namespace moe {
 namespace {
 
 constexpr int kWarpsPerCta = 8;
-constexpr int kMaxWords = kMaxRouted / 32;
 
 struct ChunkArgs {
   const int32_t* idx;
@@ -23,69 +22,75 @@ struct ChunkArgs {
   int N, k;
   int32_t* chunk_counts;     // [n_chunks, N]
   const int32_t* chunk_base; // [n_chunks, N] (scatter pass)
-  const float* gates;        // [T, k]       (scatter pass)
-  int32_t* perm;
-  int32_t* slot_pos;
-  float* gate_perm;
+  const float* gates;        // [T, k]       (scatter pass, may be null)
+  int32_t* perm;             // [R]
+  int32_t* slot_pos;         // [T, k]: rows of the token's experts, ascending expert
+  float* gate_perm;          // [R]
   unsigned* status;
 };
 
-// Pass 0 (counting) or 1 (scatter) over chunks of 32 tokens, one warp each.
+// One warp per (chunk of 32 tokens, word of 32 experts): lane l holds token
+// 32 c + l and the bits of the experts 32 w .. 32 w + 31 it selected. For each
+// expert of the word a ballot gives the tokens that chose it; a pair's rank
+// within the chunk is the popcount of the lower lanes. Pass 0 writes the
+// per-chunk counts, pass 1 places every pair.
 template <bool kScatter>
 __global__ void __launch_bounds__(32 * kWarpsPerCta) chunk_kernel(ChunkArgs a) {
-  __shared__ uint32_t bits[kWarpsPerCta][kMaxWords][32];
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int64_t c = (int64_t)blockIdx.x * kWarpsPerCta + w;
-  const int64_t n_chunks = (a.T + 31) / 32;
-  if (c >= n_chunks) return;
-  const int64_t t = c * 32 + lane;
+  const int lane = threadIdx.x & 31;
   const int W = (a.N + 31) / 32;
-  for (int i = 0; i < W; ++i) bits[w][i][lane] = 0u;
-  __syncwarp();
+  const int64_t gw = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  const int64_t n_chunks = (a.T + 31) / 32;
+  if (gw >= n_chunks * W) return;
+  const int64_t c = gw / W;
+  const int w = (int)(gw % W);
+  const int64_t t = c * 32 + lane;
   int32_t my[kMaxTopK];
-  if (t < a.T) {
-    for (int s = 0; s < a.k; ++s) {
-      int32_t e = a.idx[t * a.k + s];
-      my[s] = e;
+  uint32_t word = 0;
+#pragma unroll
+  for (int s = 0; s < kMaxTopK; ++s) {
+    my[s] = -1;
+    if (s < a.k && t < a.T) {
+      const int32_t e = a.idx[t * a.k + s];
       if (e < 0 || e >= a.N) {
-        if (!kScatter) set_status(a.status, MOE_DEV_BAD_EXPERT);
-        my[s] = -1;
+        if (!kScatter && w == 0) set_status(a.status, MOE_DEV_BAD_EXPERT);
         continue;
       }
-      uint32_t m = 1u << (e & 31);
-      if (bits[w][e >> 5][lane] & m) {
-        if (!kScatter) set_status(a.status, MOE_DEV_DUP_EXPERT);
-        my[s] = -1;
+      my[s] = e;
+      if ((e >> 5) == w) {
+        const uint32_t m = 1u << (e & 31);
+        if (word & m) {
+          if (!kScatter) set_status(a.status, MOE_DEV_DUP_EXPERT);
+          my[s] = -1;
+        }
+        word |= m;
       }
-      bits[w][e >> 5][lane] |= m;
     }
   }
-  __syncwarp();
   const uint32_t lt = (1u << lane) - 1u;
-  for (int i = 0; i < W; ++i) {
-    const uint32_t word = bits[w][i][lane];
-    int my_count = 0;
-    for (int b = 0; b < 32; ++b) {
-      const bool has = (word >> b) & 1u;
-      const uint32_t m = __ballot_sync(0xffffffffu, has);
-      if (!kScatter) {
-        if (lane == b) my_count = __popc(m);
-      } else if (has) {
-        const int e = 32 * i + b;
-        const int32_t pos = a.chunk_base[c * a.N + e] + __popc(m & lt);
-        int slot = 0;
-        for (int s = 0; s < a.k; ++s)
-          if (my[s] == e) slot = s;
-        const int32_t flat = (int32_t)(t * a.k + slot);
-        a.perm[pos] = flat;
-        a.slot_pos[flat] = pos;
-        if (a.gates) a.gate_perm[pos] = a.gates[flat];
-      }
-    }
+  int my_count = 0;
+  for (int b = 0; b < 32; ++b) {
+    const bool has = (word >> b) & 1u;
+    const uint32_t m = __ballot_sync(0xffffffffu, has);
     if (!kScatter) {
-      const int e = 32 * i + lane;
-      if (e < a.N) a.chunk_counts[c * a.N + e] = my_count;
+      if (lane == b) my_count = __popc(m);
+    } else if (has) {
+      const int e = 32 * w + b;
+      const int32_t pos = a.chunk_base[c * a.N + e] + __popc(m & lt);
+      int slot = 0, below = 0;
+#pragma unroll
+      for (int s = 0; s < kMaxTopK; ++s) {
+        if (my[s] == e) slot = s;
+        below += (my[s] >= 0 && my[s] < e) ? 1 : 0;
+      }
+      const int32_t flat = (int32_t)(t * a.k + slot);
+      a.perm[pos] = flat;
+      a.slot_pos[t * a.k + below] = pos;
+      if (a.gates) a.gate_perm[pos] = a.gates[flat];
     }
+  }
+  if (!kScatter) {
+    const int e = 32 * w + lane;
+    if (e < a.N) a.chunk_counts[c * a.N + e] = my_count;
   }
 }
 
@@ -141,8 +146,21 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a, int32_t* chunk_b
   const int tid = threadIdx.x;
   int cnt = 0;
   if (tid < a.N) {
+    // running sum over the chunks; loads are issued 8 at a time so the loop
+    // is not one L2 round trip per chunk
     int run = 0;
-    for (int64_t c = 0; c < a.n_chunks; ++c) {
+    int64_t c = 0;
+    for (; c + 8 <= a.n_chunks; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = a.chunk_counts[(c + j) * a.N + tid];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        chunk_base[(c + j) * a.N + tid] = run;
+        run += v[j];
+      }
+    }
+    for (; c < a.n_chunks; ++c) {
       int v = a.chunk_counts[c * a.N + tid];
       chunk_base[c * a.N + tid] = run;
       run += v;
@@ -154,7 +172,15 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a, int32_t* chunk_b
   if (tid < a.N) {
     a.counts[tid] = cnt;
     a.offsets[tid] = off;
-    for (int64_t c = 0; c < a.n_chunks; ++c) chunk_base[c * a.N + tid] += off;
+    int64_t c = 0;
+    for (; c + 8 <= a.n_chunks; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = chunk_base[(c + j) * a.N + tid];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) chunk_base[(c + j) * a.N + tid] = v[j] + off;
+    }
+    for (; c < a.n_chunks; ++c) chunk_base[c * a.N + tid] += off;
   }
   if (tid == 0) a.offsets[a.N] = total;
 
@@ -210,7 +236,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const TV* __restrict__ x,
 cudaError_t launch_dispatch(const Problem& p, const DispatchBuffers& db, int bm, int bn1, int bn2,
                             cudaStream_t s) {
   const int64_t n_chunks = (p.T + 31) / 32;
-  const unsigned blocks = (unsigned)((n_chunks + kWarpsPerCta - 1) / kWarpsPerCta);
+  const int64_t warps = n_chunks * ((p.N + 31) / 32);
+  const unsigned blocks = (unsigned)((warps + kWarpsPerCta - 1) / kWarpsPerCta);
   ChunkArgs ca{db.idx, p.T, p.N, p.k, db.chunk_counts, db.chunk_base, db.gates, db.perm,
                db.slot_pos, db.gate_perm, db.status};
   cudaError_t err = cudaMemsetAsync(db.slot_pos, 0xFF, (size_t)p.R * sizeof(int32_t), s);

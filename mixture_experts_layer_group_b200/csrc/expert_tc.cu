@@ -1,28 +1,43 @@
 // Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM,
-// operands staged by TMA). Two launches per layer:
+// operands staged by TMA), in "weights as M" orientation: every UMMA takes
+// 128 weight rows as its A operand (M = 128) and the group's token rows as B
+// (N = the tokens of the unit rounded up to 16, at most 256), so the MMA work
+// follows the real number of tokens per expert instead of a padded row tile.
+// A unit issues two such UMMAs per K step on one shared token tile (256
+// weight rows per unit). Two launches per layer:
 //
-//   SwiGLU GEMM  per group: g = X W1^T, u = X W3^T (one UMMA of N = 256 whose
-//                B tile stacks 128 rows of W1 over the same 128 rows of W3),
-//                epilogue h = silu(g) * u -> bf16
-//                ("Routed expert:" / "Shared expert:" steps g = x W1, u = x W3,
-//                a = g sigma(g), h = a (.) u)
-//   gate GEMM    per group: E = h W2^T (UMMA N = 256 model columns), epilogue
-//                E * G (the row's gate; 1 for the shared MLP) -> bf16 row of
-//                the token's slot ("E_i = h W2", "y_routed = sum G_i E_i")
+//   SwiGLU GEMM  unit = (group, 128 features, <= 256 tokens): half 0 is 128
+//                rows of W1, half 1 the same 128 rows of W3, so TMEM lane i
+//                holds g and u of feature i for every token column; epilogue
+//                h = silu(g) * u -> bf16
+//                ("Routed expert:" / "Shared expert:" steps g = x W1,
+//                u = x W3, a = g sigma(g), h = a (.) u)
+//   gate GEMM    unit = (group, 256 model columns, <= 256 tokens):
+//                E^T = W2 h^T; epilogue E * G (the token slot's gate; 1 for
+//                the shared MLP) -> bf16 row of the slot
+//                ("E_i = h W2", "y_routed = sum G_i E_i")
 //
 // Groups 0..N-1 are the routed experts over their expert-contiguous token
-// rows; group N is the fused shared MLP over all T tokens, scheduled in the
-// same persistent launch. A unit of work is (group, output-column tile,
-// 128-row tile); units of one group are consecutive and ordered column-tile
-// major so that concurrent CTAs share each weight tile through L2.
+// rows; group N is the fused shared MLP over all T tokens, in the same
+// persistent launch. Units of one group are consecutive, weight-tile major
+// and token-chunk minor. CTAs take units from a global counter, so the
+// chunks that share a weight tile start together (they read it once through
+// L2) and the last units balance across SMs.
 //
-// CTA roles (192 threads, one CTA per SM, persistent over units):
-//   warp 0      TMA producer (one lane): A tile 128 x 64 and B tile 256 x 64
-//               per stage, 4-stage ring of 48 KB
-//   warp 1      TMEM owner + UMMA issuer (one lane): 4 x (128 x 256 x 16)
-//               per stage into one of two 256-column fp32 accumulators
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator quadrant the warp may
-//               access, fused SwiGLU / gate, predicated row stores
+// CTA roles (192 threads, one CTA per SM, persistent):
+//   warp 0      scheduler + TMA producer (one lane): takes a unit id, hands it
+//               to the other roles through a shared-memory ring, then loads
+//               A 2 x 128 x 64 and B <= 256 x 64 bf16 per stage into a 3-stage
+//               ring of 64 KB; weights read by one unit only are evict-first
+//   warp 1      TMEM owner + UMMA issuer (one lane): 2 x 4 x (128 x N x 16)
+//               per stage. TMEM holds two buffers of 2 x 128 fp32 columns: a
+//               unit of <= 128 tokens takes one buffer (the next unit's MMAs
+//               overlap its epilogue), a larger unit takes both (2 x 256)
+//   warps 2..13 epilogue, three warps per TMEM lane quadrant taking turns on
+//               32-token blocks: each warp reads its quadrant, applies SwiGLU
+//               or the gate, transposes the 32 x 32 block through its own
+//               shared-memory tile (bf16) and writes 64-byte token-row
+//               segments; no barrier between epilogue warps per block
 // Every mbarrier wait is bounded; on a timeout the CTA records
 // MOE_DEV_WAIT_TIMEOUT, drains its own copies and MMAs (bounded again),
 // frees its tensor memory and exits.
@@ -34,35 +49,63 @@
 namespace moe {
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kBK = 64;                              // bf16 per K chunk: one 128 B swizzle row
-constexpr int kATileBytes = kTcBM * kBK * 2;         // 16 KB
-constexpr int kBTileBytes = 256 * kBK * 2;           // 32 KB
+constexpr int kStages = 3;
+constexpr int kBK = 64;                           // bf16 per K chunk: one 128 B swizzle row
+constexpr int kMaxTok = kTcBM;                    // tokens per unit (<= 256)
+constexpr int kTokBox = 32;                       // token rows per TMA box
+constexpr int kHalfBytes = 128 * kBK * 2;         // 16 KB: one M = 128 weight tile
+constexpr int kATileBytes = 2 * kHalfBytes;       // 32 KB: two of them
+constexpr int kBTileBytes = kMaxTok * kBK * 2;    // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
-constexpr int kAccCols = 256;                        // fp32 columns per accumulator
-constexpr int kTmemCols = 2 * kAccCols;
-constexpr int kThreads = 192;
-constexpr int kBarrierBytes = 256;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
-constexpr uint32_t kIdesc = idesc_bf16_f32(kTcBM, 256);
+constexpr int kBufCols = 256;                     // fp32 columns per accumulator buffer
+constexpr int kTmemCols = 2 * kBufCols;           // 2 buffers
+constexpr int kEpiWarps = 12;                     // three per TMEM lane quadrant
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kRing = 8;                          // unit ids in flight between the roles
+constexpr int kTPitch = 40;                       // bf16 per row of a warp's 32 x 32 tile (80 B)
+constexpr int kTBytes = kEpiWarps * 32 * kTPitch * 2;  // one tile per epilogue warp
+constexpr int kBarrierBytes = 512;
+constexpr int kSmemBytes = kStages * kStageBytes + kTBytes + 1024 + kBarrierBytes;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kEpiWarps % 4 == 0, "whole quadrants");
+static_assert(kMaxTok <= kBufCols && kMaxTok % kTokBox == 0, "token chunk");
 
 enum Mode : int { kSwiGLU = 0, kGateDown = 1 };
 
+// Optional per-unit timestamps (%globaltimer) of the three roles, compiled in
+// only with -DMOE_UNIT_TRACE for pipeline studies; a no-op otherwise.
+#ifdef MOE_UNIT_TRACE
+constexpr int kTraceCtas = 160, kTraceUnits = 160;
+__device__ unsigned long long g_unit_trace[2][kTraceCtas][kTraceUnits][8];
+#define MOE_TRACE_VAL(mode, unit_i, slot, value)                                        \
+  do {                                                                                 \
+    if (blockIdx.x < kTraceCtas && (unit_i) < kTraceUnits)                             \
+      g_unit_trace[mode][blockIdx.x][unit_i][slot] = (value);                          \
+  } while (0)
+#else
+#define MOE_TRACE_VAL(mode, unit_i, slot, value) \
+  do {                                           \
+    (void)(unit_i);                              \
+  } while (0)
+#endif
+#define MOE_TRACE(mode, unit_i, slot) MOE_TRACE_VAL(mode, unit_i, slot, global_timer_ns())
+
 struct TcParams {
-  CUtensorMap a_routed;   // x_perm [R, d]   | h_perm [R, F]
-  CUtensorMap a_shared;   // x [T, d]        | h_sh [T, nsF]
-  CUtensorMap b0_routed;  // W1 [N*F, d]     | W2 [N*d, F]
-  CUtensorMap b1_routed;  // W3 [N*F, d]     | unused
-  CUtensorMap b0_shared;  // Ws1 [nsF, d]    | Ws2 [d, nsF]
-  CUtensorMap b1_shared;  // Ws3 [nsF, d]    | unused
+  CUtensorMap a0_routed;  // W1 [N*F, d]      | W2 [N*d, F]
+  CUtensorMap a1_routed;  // W3 [N*F, d]      | unused
+  CUtensorMap a0_shared;  // Ws1 [nsF, d]     | Ws2 [d, nsF]
+  CUtensorMap a1_shared;  // Ws3 [nsF, d]     | unused
+  CUtensorMap b_routed;   // x_perm [R, d]    | h_perm [R, F]
+  CUtensorMap b_shared;   // x [T, d]         | h_sh [T, nsF]
   const int32_t* unit_base;  // [N + 2]: units before group g; [N + 1] = total
   const int32_t* grp_row0;   // [N + 1]
   const int32_t* grp_rows;   // [N + 1]
+  int* sched;                // unit counter, zero at launch
   int N;
   int k_routed, k_shared;        // reduction length (d | F, d | nsF)
   int cols_routed, cols_shared;  // output columns (F, nsF | d, d)
-  int b_rows_per_expert;         // rows of the stacked B per routed expert (F | d)
-  int bn;                        // output columns per tile (128 | 256)
+  int a_rows_per_expert;         // rows of the stacked weight tensor per routed expert (F | d)
+  int tile_cols;                 // output columns per unit (128 | 256)
   __nv_bfloat16* out_routed;
   int64_t ld_routed;
   __nv_bfloat16* out_shared;
@@ -72,7 +115,11 @@ struct TcParams {
 };
 
 struct Unit {
-  int g, f, m;
+  int g;        // group (N = shared MLP)
+  int f;        // output-column tile
+  int tok0;     // first token row of the chunk within the group
+  int ntok;     // tokens in the chunk (1..256)
+  int nchunks;  // chunks of the group
 };
 
 MOE_DEV Unit decode_unit(const TcParams& p, int u) {
@@ -84,34 +131,69 @@ MOE_DEV Unit decode_unit(const TcParams& p, int u) {
   }
   const int local = u - __ldg(p.unit_base + lo);
   const int rows = __ldg(p.grp_rows + lo);
-  const int mt = (rows + kTcBM - 1) / kTcBM;
-  return Unit{lo, local / mt, local % mt};
+  const int nc = (rows + kMaxTok - 1) / kMaxTok;
+  Unit un;
+  un.g = lo;
+  un.f = local / nc;
+  un.tok0 = (local % nc) * kMaxTok;
+  const int left = rows - un.tok0;
+  un.ntok = left < kMaxTok ? left : kMaxTok;
+  un.nchunks = nc;
+  return un;
 }
+
+// Accumulator placement. A unit of <= 128 tokens takes one buffer (its two
+// halves at columns base and base + 128); a larger unit takes both buffers
+// (halves at columns 0 and 256). The MMA issuer and every epilogue thread
+// replay the same sequence, so they agree on every placement.
+struct AccPlan {
+  uint32_t next = 0;
+  MOE_DEV void place(int ntok, uint32_t& mask, uint32_t& base, uint32_t& stride) const {
+    if (ntok > kBufCols / 2) {
+      mask = 3u;
+      base = 0;
+      stride = kBufCols;
+    } else {
+      mask = 1u << next;
+      base = next * kBufCols;
+      stride = kBufCols / 2;
+    }
+  }
+  MOE_DEV void advance(int ntok) { next = ntok > kBufCols / 2 ? 0u : next ^ 1u; }
+};
 
 struct Shared {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
+  uint64_t ring_full[kRing];
+  uint64_t ring_empty[kRing];
   uint64_t drained;
+  int ring[kRing];
+  int epi_unit[2];    // the epilogue leader's unit for the 4 epilogue warps
   uint32_t tmem_base;
   int abort_flag;
   uint32_t consumed;  // stage fills the MMA issuer observed complete
 };
 
-// Stores 32 consecutive values of one row as bf16 (16-byte stores), or the
-// first ncols of them at a ragged right edge.
-MOE_DEV void store_cols(__nv_bfloat16* dst, int ncols, const float (&v)[32]) {
+// Barrier among the epilogue warps only (id 1; id 0 is __syncthreads).
+MOE_DEV void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
+
+MOE_DEV int load_volatile(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
+
+// Writes one 64-byte token-row segment (32 bf16 from the transpose tile),
+// or the first ncols of it at a ragged right edge.
+MOE_DEV void store_row32(__nv_bfloat16* dst, int ncols, const uint4 (&v)[4]) {
   if (ncols >= 32) {
     uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      d4[i] = make_uint4(pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                         pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+    for (int c = 0; c < 4; ++c) d4[c] = v[c];
   } else {
+    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(v);
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < ncols) dst[j] = __float2bfloat16_rn(v[j]);
+    for (int c = 0; c < 32; ++c)
+      if (c < ncols) dst[c] = e[c];
   }
 }
 
@@ -119,7 +201,8 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Shared& sh = *reinterpret_cast<Shared*>(smem + kStages * kStageBytes);
+  float* tiles = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+  Shared& sh = *reinterpret_cast<Shared*>(smem + kStages * kStageBytes + kTBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -132,7 +215,11 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.acc_full[b], 1);
-      mbar_init(&sh.acc_empty[b], 4);
+      mbar_init(&sh.acc_empty[b], kEpiWarps);
+    }
+    for (int q = 0; q < kRing; ++q) {
+      mbar_init(&sh.ring_full[q], 1);
+      mbar_init(&sh.ring_empty[q], 2);  // MMA issuer + epilogue leader
     }
     mbar_init(&sh.drained, 1);
     sh.abort_flag = 0;
@@ -140,9 +227,9 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&p.a_routed);
-    tma_prefetch_desc(&p.b0_routed);
-    if (MODE == kSwiGLU) tma_prefetch_desc(&p.b1_routed);
+    tma_prefetch_desc(&p.a0_routed);
+    tma_prefetch_desc(&p.b_routed);
+    if (MODE == kSwiGLU) tma_prefetch_desc(&p.a1_routed);
   }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, kTmemCols);
@@ -156,20 +243,40 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
 
   uint32_t fills = 0;  // producer: stage fills issued
   if (warp == 0) {
-    // ------------------------------------------------------------ producer --
+    // ------------------------------------------------- scheduler + producer --
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();  // weights: each tile is streamed once
-      for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+      // a weight tile read by one unit only is streamed once: evict it first;
+      // tiles shared by the chunks of a large group stay at normal priority
+      const uint64_t pol_once = policy_evict_first();
+      const uint64_t pol_shared = policy_evict_normal();
+      bool ok = true;
+      for (int i = 0;; ++i) {
+        const int q = i % kRing;
+        if (!mbar_wait_bounded(&sh.ring_empty[q], ((i / kRing) & 1) ^ 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        int u = atomicAdd(p.sched, 1);
+        if (u >= total_units) u = -1;
+        sh.ring[q] = u;
+        mbar_arrive(&sh.ring_full[q]);
+        if (u < 0) break;
         const Unit un = decode_unit(p, u);
         const bool shared = un.g == p.N;
         const int K = shared ? p.k_shared : p.k_routed;
         const int nk = (K + kBK - 1) / kBK;
-        const int rowA = __ldg(p.grp_row0 + un.g) + un.m * kTcBM;
-        const int rowB = (shared ? 0 : un.g * p.b_rows_per_expert) + un.f * p.bn;
-        const CUtensorMap* ta = shared ? &p.a_shared : &p.a_routed;
-        const CUtensorMap* tb0 = shared ? &p.b0_shared : &p.b0_routed;
-        const CUtensorMap* tb1 = shared ? &p.b1_shared : &p.b1_routed;
-        bool ok = true;
+        const int nbox = (un.ntok + kTokBox - 1) / kTokBox;
+        const uint32_t tx = kATileBytes + nbox * (kTokBox * kBK * 2);
+        const int rowA = (shared ? 0 : un.g * p.a_rows_per_expert) + un.f * p.tile_cols;
+        const int rowB = __ldg(p.grp_row0 + un.g) + un.tok0;
+        const CUtensorMap* ta0 = shared ? &p.a0_shared : &p.a0_routed;
+        const CUtensorMap* ta1 = MODE == kSwiGLU ? (shared ? &p.a1_shared : &p.a1_routed) : ta0;
+        const int rowA1 = MODE == kSwiGLU ? rowA : rowA + 128;  // W3 rows | next 128 W2 rows
+        const CUtensorMap* tb = shared ? &p.b_shared : &p.b_routed;
+        const uint64_t pol = un.nchunks == 1 ? pol_once : pol_shared;
+        MOE_TRACE(MODE, i, 0);
+        MOE_TRACE_VAL(MODE, i, 7, (unsigned long long)un.ntok | ((unsigned long long)un.tok0 << 16) |
+                                      ((unsigned long long)un.g << 32) | ((unsigned long long)un.f << 48));
         for (int kc = 0; kc < nk; ++kc, ++fills) {
           const uint32_t s = fills % kStages, ph = (fills / kStages) & 1u;
           if (!mbar_wait_bounded(&sh.empty[s], ph ^ 1u, abort_flag)) {
@@ -178,20 +285,18 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           }
           uint8_t* a_dst = smem + s * kStageBytes;
           uint8_t* b_dst = a_dst + kATileBytes;
-          mbar_arrive_expect_tx(&sh.full[s], kStageBytes);
-          tma_load_2d(a_dst, ta, &sh.full[s], kc * kBK, rowA);
-          if (MODE == kSwiGLU) {
-            tma_load_2d_hint(b_dst, tb0, &sh.full[s], kc * kBK, rowB, pol_w);
-            tma_load_2d_hint(b_dst + kBTileBytes / 2, tb1, &sh.full[s], kc * kBK, rowB, pol_w);
-          } else {
-            tma_load_2d_hint(b_dst, tb0, &sh.full[s], kc * kBK, rowB, pol_w);
-          }
+          mbar_arrive_expect_tx(&sh.full[s], tx);
+          tma_load_2d_hint(a_dst, ta0, &sh.full[s], kc * kBK, rowA, pol);
+          tma_load_2d_hint(a_dst + kHalfBytes, ta1, &sh.full[s], kc * kBK, rowA1, pol);
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(b_dst + b * (kTokBox * kBK * 2), tb, &sh.full[s], kc * kBK, rowB + b * kTokBox);
         }
-        if (!ok) {
-          *abort_flag = 1;
-          set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
-          break;
-        }
+        MOE_TRACE(MODE, i, 1);
+        if (!ok) break;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
       }
     }
     __syncwarp();
@@ -199,19 +304,35 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
     // ---------------------------------------------------------- MMA issuer --
     if (lane == 0) {
       uint32_t consumed = 0;
-      int i = 0;
+      uint32_t uses[2] = {0u, 0u};
+      AccPlan plan;
       bool ok = true;
-      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++i) {
-        const Unit un = decode_unit(p, u);
-        const int K = un.g == p.N ? p.k_shared : p.k_routed;
-        const int nk = (K + kBK - 1) / kBK;
-        const uint32_t buf = i & 1, aph = (i >> 1) & 1;
-        if (!mbar_wait_bounded(&sh.acc_empty[buf], aph ^ 1u, abort_flag)) {
+      for (int i = 0; ok; ++i) {
+        const int q = i % kRing;
+        if (!mbar_wait_bounded(&sh.ring_full[q], (i / kRing) & 1, abort_flag)) {
           ok = false;
           break;
         }
+        const int u = load_volatile(&sh.ring[q]);
+        mbar_arrive(&sh.ring_empty[q]);
+        if (u < 0) break;
+        const Unit un = decode_unit(p, u);
+        const int K = un.g == p.N ? p.k_shared : p.k_routed;
+        const int nk = (K + kBK - 1) / kBK;
+        const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)((un.ntok + 15) & ~15));
+        uint32_t mask, base, stride;
+        plan.place(un.ntok, mask, base, stride);
+        plan.advance(un.ntok);
+        MOE_TRACE(MODE, i, 2);
+        for (int b = 0; b < 2 && ok; ++b)
+          if ((mask >> b) & 1u) {
+            ok = mbar_wait_bounded(&sh.acc_empty[b], (uses[b] & 1u) ^ 1u, abort_flag);
+            ++uses[b];
+          }
+        if (!ok) break;
+        MOE_TRACE(MODE, i, 3);
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * kAccCols;
+        const uint32_t d0 = tmem_base + base, d1 = tmem_base + base + stride;
         for (int kc = 0; kc < nk; ++kc) {
           const uint32_t s = consumed % kStages, ph = (consumed / kStages) & 1u;
           if (!mbar_wait_bounded(&sh.full[s], ph, abort_flag)) {
@@ -224,12 +345,17 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           const uint32_t b_addr = a_addr + kATileBytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            umma_bf16(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
-                      kIdesc, (kc | kk) != 0);
+            const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32);
+            umma_bf16(d0, smem_desc_sw128(a_addr + kk * 32), bdesc, idesc, (kc | kk) != 0);
+            umma_bf16(d1, smem_desc_sw128(a_addr + kHalfBytes + kk * 32), bdesc, idesc, (kc | kk) != 0);
           }
           umma_commit(&sh.empty[s]);
         }
-        if (ok) umma_commit(&sh.acc_full[buf]);
+        if (ok) {
+          if (mask & 1u) umma_commit(&sh.acc_full[0]);
+          if (mask & 2u) umma_commit(&sh.acc_full[1]);
+        }
+        MOE_TRACE(MODE, i, 4);
       }
       if (!ok) {
         *abort_flag = 1;
@@ -244,56 +370,104 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue --
-    const int q = warp & 3;          // TMEM lane quadrant this warp may access
-    const int r = q * 32 + lane;     // row of the 128-row tile
-    int i = 0;
-    for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++i) {
-      const Unit un = decode_unit(p, u);
-      const bool shared = un.g == p.N;
-      const uint32_t buf = i & 1, aph = (i >> 1) & 1;
-      if (!mbar_wait_bounded(&sh.acc_full[buf], aph, abort_flag)) {
-        *abort_flag = 1;
-        set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
-        break;
-      }
-      tc_fence_after();
-      const int row_in_group = un.m * kTcBM + r;
-      const bool valid = row_in_group < __ldg(p.grp_rows + un.g);
-      const int64_t row = shared ? row_in_group : (int64_t)__ldg(p.grp_row0 + un.g) + row_in_group;
-      __nv_bfloat16* out = shared ? p.out_shared + row * p.ld_shared : p.out_routed + row * p.ld_routed;
-      const int cols = shared ? p.cols_shared : p.cols_routed;
-      const int col0 = un.f * p.bn;
-      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + buf * kAccCols;
-      if (MODE == kSwiGLU) {
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t gv[32], uv[32];
-          tmem_ld32(t_row + c, gv);
-          tmem_ld32(t_row + 128 + c, uv);
-          tmem_wait_ld();
-          float h[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) h[j] = silu_f32(__uint_as_float(gv[j])) * __uint_as_float(uv[j]);
-          const int ncols = cols - (col0 + c);
-          if (valid && ncols > 0) store_cols(out + col0 + c, ncols, h);
+    const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+    const int ew = warp - 2;                 // epilogue warp: its transpose tile
+    const int sub = ew >> 2;                 // which of the quadrant's warps
+    __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(tiles) + ew * 32 * kTPitch;
+    const bool leader = threadIdx.x == 64;
+    uint32_t uses[2] = {0u, 0u};
+    AccPlan plan;
+    for (int i = 0;; ++i) {
+      // the leader takes the next unit and waits for its accumulator(s); the
+      // epilogue warps then agree on the outcome and all run the unit or all leave
+      if (leader) {
+        int u = -2;
+        const int qr = i % kRing;
+        if (mbar_wait_bounded(&sh.ring_full[qr], (i / kRing) & 1, abort_flag)) {
+          u = load_volatile(&sh.ring[qr]);
+          mbar_arrive(&sh.ring_empty[qr]);
+          if (u >= 0) {
+            const Unit un = decode_unit(p, u);
+            uint32_t mask, base, stride;
+            plan.place(un.ntok, mask, base, stride);
+            bool ok = true;
+            for (int b = 0; b < 2 && ok; ++b)
+              if ((mask >> b) & 1u) ok = mbar_wait_bounded(&sh.acc_full[b], uses[b] & 1u, abort_flag);
+            if (!ok) u = -2;
+          }
         }
-      } else {
-        const float gate = shared ? 1.0f : (valid ? __ldg(p.gate_perm + row) : 0.f);
+        if (u == -2) {
+          *abort_flag = 1;
+          set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
+        }
+        sh.epi_unit[i & 1] = u;
+      }
+      epi_sync();
+      const int u = load_volatile(&sh.epi_unit[i & 1]);
+      if (u < 0) break;
+      const Unit un = decode_unit(p, u);
+      uint32_t mask, base, stride;
+      plan.place(un.ntok, mask, base, stride);
+      plan.advance(un.ntok);
+      uses[0] += mask & 1u;
+      uses[1] += (mask >> 1) & 1u;
+      if (leader) MOE_TRACE(MODE, i, 5);
+      tc_fence_after();
+      const bool shared = un.g == p.N;
+      const int64_t row_base = shared ? (int64_t)un.tok0 : (int64_t)__ldg(p.grp_row0 + un.g) + un.tok0;
+      __nv_bfloat16* out_base = shared ? p.out_shared : p.out_routed;
+      const int64_t ld = shared ? p.ld_shared : p.ld_routed;
+      const int cols = shared ? p.cols_shared : p.cols_routed;
+      const uint32_t t_q = tmem_base + ((uint32_t)(q * 32) << 16) + base;
+      constexpr int kHalves = MODE == kSwiGLU ? 1 : 2;
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(t_row + c, v);
-          tmem_wait_ld();
-          float o[32];
+      for (int hh = 0; hh < kHalves; ++hh) {
+        // this warp's 32 output columns of the unit
+        const int c0 = un.f * p.tile_cols + (MODE == kSwiGLU ? 0 : 128 * hh) + 32 * q;
+#pragma unroll 1
+        for (int j0 = 32 * sub; j0 < un.ntok; j0 += 32 * (kEpiWarps / 4)) {
+          const int tok = j0 + lane;
+          const int64_t row = row_base + tok;
+          // gate of this lane's token, spread to the column-owning lanes below
+          float my_gate = 1.0f;
+          if (MODE == kGateDown && !shared && tok < un.ntok) my_gate = __ldg(p.gate_perm + row);
+          float v[32];
+          {
+            uint32_t a[32];
+            tmem_ld32(t_q + hh * stride + j0, a);
+            if (MODE == kSwiGLU) {
+              uint32_t b[32];
+              tmem_ld32(t_q + stride + j0, b);  // u of the same feature
+              tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(v[j]) * gate;
-          const int ncols = cols - (col0 + c);
-          if (valid && ncols > 0) store_cols(out + col0 + c, ncols, o);
+              for (int j = 0; j < 32; ++j) {
+                const float g = __uint_as_float(a[j]);
+                v[j] = __fdividef(g, 1.0f + __expf(-g)) * __uint_as_float(b[j]);
+              }
+            } else {
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]) * __shfl_sync(0xffffffffu, my_gate, j);
+            }
+          }
+          // transpose through this warp's tile: lane = column -> lane = token
+#pragma unroll
+          for (int j = 0; j < 32; ++j) tile[j * kTPitch + lane] = __float2bfloat16_rn(v[j]);
+          __syncwarp();
+          uint4 rowv[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) rowv[c] = *reinterpret_cast<const uint4*>(tile + lane * kTPitch + 8 * c);
+          __syncwarp();
+          if (tok < un.ntok) store_row32(out_base + row * ld + c0, cols - c0, rowv);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
+      if (leader) MOE_TRACE(MODE, i, 6);
+      if (lane == 0) {
+        if (mask & 1u) mbar_arrive(&sh.acc_empty[0]);
+        if (mask & 2u) mbar_arrive(&sh.acc_empty[1]);
+      }
     }
   }
 
@@ -370,26 +544,30 @@ cudaError_t launch_one(const TcParams& prm, int grid, cudaStream_t s) {
 cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStream_t s,
                                    cudaEvent_t between) {
   const int sms = device_sm_count();
-  const int64_t mt_bound = (p.R + kTcBM - 1) / kTcBM + p.N + (p.ns > 0 ? (p.T + kTcBM - 1) / kTcBM : 0);
+  cudaError_t err0 = cudaMemsetAsync(a.sched, 0, 2 * sizeof(int), s);
+  if (err0 != cudaSuccess) return err0;
+  const int64_t chunks_bound =
+      (p.R + kMaxTok - 1) / kMaxTok + p.N + (p.ns > 0 ? (p.T + kMaxTok - 1) / kMaxTok : 0);
 
   TcParams g1{};
-  bool ok = make_tmap(&g1.a_routed, a.x_perm, (uint64_t)p.R, p.d, kTcBM) &&
-            make_tmap(&g1.a_shared, p.ns ? a.x : nullptr, (uint64_t)p.T, p.d, kTcBM) &&
-            make_tmap(&g1.b0_routed, a.W1, (uint64_t)p.N * p.F, p.d, 128) &&
-            make_tmap(&g1.b1_routed, a.W3, (uint64_t)p.N * p.F, p.d, 128) &&
-            make_tmap(&g1.b0_shared, a.Ws1, (uint64_t)p.nsF, p.d, 128) &&
-            make_tmap(&g1.b1_shared, a.Ws3, (uint64_t)p.nsF, p.d, 128);
+  bool ok = make_tmap(&g1.a0_routed, a.W1, (uint64_t)p.N * p.F, p.d, 128) &&
+            make_tmap(&g1.a1_routed, a.W3, (uint64_t)p.N * p.F, p.d, 128) &&
+            make_tmap(&g1.a0_shared, a.Ws1, (uint64_t)p.nsF, p.d, 128) &&
+            make_tmap(&g1.a1_shared, a.Ws3, (uint64_t)p.nsF, p.d, 128) &&
+            make_tmap(&g1.b_routed, a.x_perm, (uint64_t)p.R, p.d, kTokBox) &&
+            make_tmap(&g1.b_shared, p.ns ? a.x : nullptr, (uint64_t)p.T, p.d, kTokBox);
   if (!ok) return cudaErrorInvalidValue;
   g1.unit_base = a.unit_base1;
   g1.grp_row0 = a.grp_row0;
   g1.grp_rows = a.grp_rows;
+  g1.sched = a.sched;
   g1.N = p.N;
   g1.k_routed = p.d;
   g1.k_shared = p.d;
   g1.cols_routed = p.F;
   g1.cols_shared = p.nsF;
-  g1.b_rows_per_expert = p.F;
-  g1.bn = kTcBN1;
+  g1.a_rows_per_expert = p.F;
+  g1.tile_cols = kTcBN1;
   g1.out_routed = (__nv_bfloat16*)a.h_perm;
   g1.ld_routed = p.F;
   g1.out_shared = (__nv_bfloat16*)a.h_sh;
@@ -397,38 +575,49 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g1.gate_perm = nullptr;
   g1.status = a.status;
   const int64_t max_cols1 = p.F > p.nsF ? p.F : p.nsF;
-  const int64_t units1 = mt_bound * ((max_cols1 + kTcBN1 - 1) / kTcBN1);
+  const int64_t units1 = chunks_bound * ((max_cols1 + kTcBN1 - 1) / kTcBN1);
   const int grid1 = (int)(units1 < sms ? units1 : sms);
   cudaError_t err = launch_one<kSwiGLU>(g1, grid1 > 0 ? grid1 : 1, s);
   if (err == cudaSuccess && between) err = cudaEventRecord(between, s);
   if (err != cudaSuccess) return err;
 
   TcParams g2{};
-  ok = make_tmap(&g2.a_routed, a.h_perm, (uint64_t)p.R, p.F, kTcBM) &&
-       make_tmap(&g2.a_shared, p.ns ? a.h_sh : nullptr, (uint64_t)p.T, p.nsF, kTcBM) &&
-       make_tmap(&g2.b0_routed, a.W2, (uint64_t)p.N * p.d, p.F, 256) &&
-       make_tmap(&g2.b0_shared, a.Ws2, (uint64_t)p.d, p.nsF, 256);
+  ok = make_tmap(&g2.a0_routed, a.W2, (uint64_t)p.N * p.d, p.F, 128) &&
+       make_tmap(&g2.a0_shared, a.Ws2, (uint64_t)p.d, p.nsF, 128) &&
+       make_tmap(&g2.b_routed, a.h_perm, (uint64_t)p.R, p.F, kTokBox) &&
+       make_tmap(&g2.b_shared, p.ns ? a.h_sh : nullptr, (uint64_t)p.T, p.nsF, kTokBox);
   if (!ok) return cudaErrorInvalidValue;
   g2.unit_base = a.unit_base2;
   g2.grp_row0 = a.grp_row0;
   g2.grp_rows = a.grp_rows;
+  g2.sched = a.sched + 1;
   g2.N = p.N;
   g2.k_routed = p.F;
   g2.k_shared = p.nsF;
   g2.cols_routed = p.d;
   g2.cols_shared = p.d;
-  g2.b_rows_per_expert = p.d;
-  g2.bn = kTcBN2;
+  g2.a_rows_per_expert = p.d;
+  g2.tile_cols = kTcBN2;
   g2.out_routed = (__nv_bfloat16*)a.y_rows;
   g2.ld_routed = p.d;
   g2.out_shared = (__nv_bfloat16*)a.y_rows + p.R * (int64_t)p.d;
   g2.ld_shared = p.d;
   g2.gate_perm = a.gate_perm;
   g2.status = a.status;
-  const int64_t nt2 = (p.d + kTcBN2 - 1) / kTcBN2;
-  const int64_t units2 = mt_bound * nt2;
+  const int64_t units2 = chunks_bound * ((p.d + kTcBN2 - 1) / kTcBN2);
   const int grid2 = (int)(units2 < sms ? units2 : sms);
   return launch_one<kGateDown>(g2, grid2 > 0 ? grid2 : 1, s);
 }
 
 }  // namespace moe
+
+#ifdef MOE_UNIT_TRACE
+// Copies the unit trace ([2][kTraceCtas][kTraceUnits][8] u64) to host memory
+// and clears it (trace builds only).
+extern "C" MOE_API int moe_unit_trace_read(void* host_dst) {
+  cudaError_t e = cudaMemcpyFromSymbol(host_dst, moe::g_unit_trace, sizeof(moe::g_unit_trace));
+  if (e != cudaSuccess) return (int)e;
+  static unsigned long long zeros[2 * moe::kTraceCtas * moe::kTraceUnits * 8];
+  return (int)cudaMemcpyToSymbol(moe::g_unit_trace, zeros, sizeof(zeros));
+}
+#endif

@@ -10,11 +10,14 @@
 
 namespace moe {
 
-// Tile sizes of the tensor-core grouped GEMMs (rows x columns of one output
-// tile) and of the fp32 SIMT grouped GEMMs.
-constexpr int kTcBM = 128;      // token rows per tile (UMMA M)
-constexpr int kTcBN1 = 128;     // SwiGLU GEMM: features per tile (g and u: UMMA N = 256)
-constexpr int kTcBN2 = 256;     // down-projection GEMM: model columns per tile (UMMA N)
+// Tile sizes of the tensor-core grouped GEMMs: a unit covers at most
+// kTcBM token rows of one group (UMMA N) and kTcBN1 SwiGLU features (two
+// UMMAs of M = 128, each 64 W1 rows stacked over 64 W3 rows) or kTcBN2 model
+// columns of the down projection (two UMMAs of M = 128). The fp32 SIMT GEMMs
+// use 64 x 64 tiles.
+constexpr int kTcBM = 256;
+constexpr int kTcBN1 = 128;
+constexpr int kTcBN2 = 256;
 constexpr int kSimtBM = 64;
 constexpr int kSimtBN = 64;
 constexpr int kChunkTokens = 32;  // dispatch: tokens per warp chunk
@@ -33,7 +36,7 @@ struct Problem {
 
 // Byte offsets of every workspace region (all 256-byte aligned).
 struct Layout {
-  size_t status, logits, idx, gates, chunk_counts, chunk_base, counts, offsets;
+  size_t status, sched, logits, idx, gates, chunk_counts, chunk_base, counts, offsets;
   size_t grp_row0, grp_rows, unit_base1, unit_base2, perm, slot_pos, gate_perm;
   size_t x_perm, h_perm, h_sh, y_rows, x_stage, y_stage;
   size_t total, total_host;
@@ -54,15 +57,21 @@ struct DispatchBuffers {
   int32_t* unit_base1;
   int32_t* unit_base2;
   int32_t* perm;
-  int32_t* slot_pos;
+  int32_t* slot_pos;   // [T, k]: permuted rows of the token's experts, ascending expert
   float* gate_perm;
   const float* gates;
   unsigned* status;
 };
 
-// Router: logits (SIMT fp32) then selection.
+// Router: logits (SIMT fp32) then selection. With router_scratch_bytes(p)
+// bytes of logits scratch the router uses router_k_splits(p) K ranges; with
+// less (at least T * N * 4) it uses as many as fit.
+constexpr int kRouterTargetSms = 148;
+int router_k_splits(const Problem& p);
+size_t router_scratch_bytes(const Problem& p);
 cudaError_t launch_router(const Problem& p, const void* x, const void* W_r, const float* b,
-                          float* logits, int32_t* idx, float* gates, cudaStream_t s);
+                          float* logits, size_t logits_bytes, int32_t* idx, float* gates,
+                          cudaStream_t s);
 
 // Histogram / scan / scatter; bm, bn1, bn2 select the GEMM tile grid that
 // the unit tables describe.
@@ -91,6 +100,7 @@ struct GemmArgs {
   const int32_t* unit_base2;
   const float* gate_perm;
   unsigned* status;
+  int* sched;           // [2] unit counters of the two tensor-core launches
 };
 
 // Tensor-core (bf16) expert GEMMs: SwiGLU projection then gated down
@@ -101,9 +111,10 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
 cudaError_t launch_expert_gemms_simt(const Problem& p, const GemmArgs& a, cudaStream_t s,
                                      cudaEvent_t between);
 
-// y[t] = sum over slots (ascending expert) of y_rows[slot_pos] + y_rows[R + t]
-cudaError_t launch_combine(const Problem& p, const void* y_rows, const int32_t* slot_pos,
-                           const int32_t* idx, void* y, cudaStream_t s);
+// y[t] = sum over the token's rows slot_pos[t, 0..k) (ascending expert) of
+// y_rows, plus the shared row y_rows[R + t]
+cudaError_t launch_combine(const Problem& p, const void* y_rows, const int32_t* slot_pos, void* y,
+                           cudaStream_t s);
 
 int device_sm_count();
 

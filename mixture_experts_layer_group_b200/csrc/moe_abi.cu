@@ -98,7 +98,8 @@ Layout make_layout(const Problem& p) {
   const int64_t T = p.T, N = p.N, R = p.R;
   L.n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
   L.status = take(256);
-  L.logits = take((size_t)T * N * 4);
+  L.sched = take(256);
+  L.logits = take(router_scratch_bytes(p));
   L.idx = take((size_t)R * 4);
   L.gates = take((size_t)R * 4);
   L.chunk_counts = take((size_t)L.n_chunks * N * 4);
@@ -138,7 +139,7 @@ moe_status check_ws(const Layout& L, void* ws, size_t ws_bytes, size_t need) {
 
 moe_status run_router(const Problem& p, const Layout& L, const void* x, const void* W_r,
                       const float* b, int32_t* idx, float* gates, void* ws, cudaStream_t s) {
-  cudaError_t e = launch_router(p, x, W_r, b, at<float>(ws, L.logits), idx, gates, s);
+  cudaError_t e = launch_router(p, x, W_r, b, at<float>(ws, L.logits), router_scratch_bytes(p), idx, gates, s);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
@@ -200,11 +201,12 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
   ga.unit_base2 = db.unit_base2;
   ga.gate_perm = db.gate_perm;
   ga.status = db.status;
+  ga.sched = at<int>(ws, L.sched);
   e = tc ? launch_expert_gemms_tc(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr)
          : launch_expert_gemms_simt(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr);
   if (e == cudaSuccess) e = mark_stage(5, s);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = launch_combine(p, ga.y_rows, db.slot_pos, idx, y, s);
+  e = launch_combine(p, ga.y_rows, db.slot_pos, y, s);
   if (e == cudaSuccess) e = mark_stage(6, s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (idx_out) {

@@ -16,7 +16,8 @@
 namespace moe {
 namespace {
 
-// Largest scratch a call may use: T * n_routed * 4 bytes of logits.
+// Largest scratch a call may use: the router's fp32 logits, T * n_routed * 4
+// bytes (the router splits its reduction only as far as the array allows).
 constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB
 constexpr int kMaxDevices = 64;
 
@@ -64,7 +65,7 @@ extern "C" moe_status moe_route_noalloc(const moe_cfg* cfg, int64_t T, const voi
   void* scratch = nullptr;
   cudaError_t e = scratch_address(&scratch);
   if (e == cudaSuccess)
-    e = launch_router(p, x, W_r, b, static_cast<float*>(scratch), topk_idx, gates,
+    e = launch_router(p, x, W_r, b, static_cast<float*>(scratch), kNoallocScratchBytes, topk_idx, gates,
                       static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     record_cuda_error(e);

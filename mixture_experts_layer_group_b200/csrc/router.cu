@@ -6,7 +6,10 @@
 // Logits are accumulated in fp32 over 32-element K chunks and carried across
 // chunks in fp64, which keeps the logit error near 1e-7 at d = 7168 (a plain
 // fp32 running sum is an order of magnitude worse and would turn near-ties
-// into routing differences). bf16 products are exact in fp32.
+// into routing differences). bf16 products are exact in fp32. When the
+// token count alone gives too few CTAs (decode), K is split into S ranges
+// whose partial logits the selection kernel adds in a fixed order, so the
+// result stays deterministic.
 #include <cfloat>
 #include <cmath>
 
@@ -27,11 +30,12 @@ struct Vec16 {
   static constexpr int kElems = 16 / sizeof(TIn);
 };
 
-// Loads 16 bytes of row `row` at column k (zero outside [0, rows) x [0, d)).
+// Loads 16 bytes of row `row` (row pitch d) at column k (zero outside
+// [0, rows) x [0, k_end)).
 template <typename TIn>
-MOE_DEV void load_vec(const TIn* base, int64_t rows, int d, int64_t row, int k, float* out) {
+MOE_DEV void load_vec(const TIn* base, int64_t rows, int k_end, int d, int64_t row, int k, float* out) {
   constexpr int E = Vec16<TIn>::kElems;
-  if (row < rows && k < d) {
+  if (row < rows && k < k_end) {
     uint4 v = *reinterpret_cast<const uint4*>(base + row * (int64_t)d + k);
     if constexpr (sizeof(TIn) == 2) {
       const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&v);
@@ -54,7 +58,7 @@ MOE_DEV void load_vec(const TIn* base, int64_t rows, int d, int64_t row, int k, 
 template <typename TIn>
 __global__ void __launch_bounds__(kLThreads) router_logits_kernel(const TIn* __restrict__ x,
                                                                   const TIn* __restrict__ W,
-                                                                  int64_t T, int N, int d,
+                                                                  int64_t T, int N, int d, int k_len,
                                                                   float* __restrict__ logits) {
   constexpr int E = Vec16<TIn>::kElems;          // elements per 16-byte vector
   constexpr int kVecPerRow = kLBK / E;           // vectors per row per chunk
@@ -69,6 +73,10 @@ __global__ void __launch_bounds__(kLThreads) router_logits_kernel(const TIn* __r
   const int tx = tid & 15, ty = tid >> 4;
   const int64_t t0 = (int64_t)blockIdx.y * kLBT;
   const int64_t e0 = (int64_t)blockIdx.x * kLBN;
+  // this CTA's K range [k_begin, k_end) and its partial-logit plane
+  const int k_begin = blockIdx.z * k_len;
+  const int k_end = min(d, k_begin + k_len);
+  logits += (int64_t)blockIdx.z * T * N;
 
   float xr[kLoads][E], wr[kLoads][E];
   auto fetch = [&](int kbase) {
@@ -76,8 +84,8 @@ __global__ void __launch_bounds__(kLThreads) router_logits_kernel(const TIn* __r
     for (int i = 0; i < kLoads; ++i) {
       int v = tid + i * kLThreads;
       int row = v / kVecPerRow, kv = (v % kVecPerRow) * E;
-      load_vec<TIn>(x, T, d, t0 + row, kbase + kv, xr[i]);
-      load_vec<TIn>(W, N, d, e0 + row, kbase + kv, wr[i]);
+      load_vec<TIn>(x, T, k_end, d, t0 + row, kbase + kv, xr[i]);
+      load_vec<TIn>(W, N, k_end, d, e0 + row, kbase + kv, wr[i]);
     }
   };
   auto stash = [&]() {
@@ -101,13 +109,13 @@ __global__ void __launch_bounds__(kLThreads) router_logits_kernel(const TIn* __r
 #pragma unroll
     for (int b = 0; b < 4; ++b) total[a][b] = 0.0;
 
-  const int nk = (d + kLBK - 1) / kLBK;
-  fetch(0);
+  const int nk = (k_end - k_begin + kLBK - 1) / kLBK;
+  fetch(k_begin);
   for (int kc = 0; kc < nk; ++kc) {
     __syncthreads();
     stash();
     __syncthreads();
-    if (kc + 1 < nk) fetch((kc + 1) * kLBK);
+    if (kc + 1 < nk) fetch(k_begin + (kc + 1) * kLBK);
     float acc[4][4];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
@@ -191,7 +199,8 @@ MOE_DEV void merge_top2(float& a1, float& a2, float b1, float b2) {
 }
 
 struct SelectArgs {
-  const float* logits;
+  const float* logits;  // [S, T, N] partial logits
+  int S;
   const float* bias;
   int64_t T;
   int N, k, G, TG, score_fn, group_score, normalize;
@@ -213,7 +222,13 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
 #pragma unroll
   for (int j = 0; j < V; ++j) {
     int e = 32 * j + lane;
-    s[j] = e < N ? zrow[e] : -INFINITY;
+    if (e < N) {
+      float z = zrow[e];
+      for (int sp = 1; sp < a.S; ++sp) z += zrow[(int64_t)sp * a.T * N + e];  // fixed order
+      s[j] = z;
+    } else {
+      s[j] = -INFINITY;
+    }
   }
   if (a.score_fn == MOE_SOFTMAX) {
     float m = -INFINITY;
@@ -306,19 +321,40 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
 
 }  // namespace
 
+int router_k_splits(const Problem& p) {
+  // enough CTAs to fill the SMs twice, each split keeping >= 4 K chunks
+  const int64_t base = (int64_t)((p.N + kLBN - 1) / kLBN) * ((p.T + kLBT - 1) / kLBT);
+  int64_t S = base > 0 ? (2 * (int64_t)kRouterTargetSms) / base : 1;
+  const int64_t by_k = p.d / (4 * kLBK);
+  if (S > by_k) S = by_k;
+  if (S > 16) S = 16;
+  return S < 1 ? 1 : (int)S;
+}
+
+size_t router_scratch_bytes(const Problem& p) {
+  return (size_t)router_k_splits(p) * (size_t)p.T * (size_t)p.N * sizeof(float);
+}
+
 cudaError_t launch_router(const Problem& p, const void* x, const void* W_r, const float* b,
-                          float* logits, int32_t* idx, float* gates, cudaStream_t s) {
-  dim3 grid((unsigned)((p.N + kLBN - 1) / kLBN), (unsigned)((p.T + kLBT - 1) / kLBT));
+                          float* logits, size_t logits_bytes, int32_t* idx, float* gates,
+                          cudaStream_t s) {
+  // as many K splits as router_k_splits(p) asks for and the scratch can hold
+  const size_t plane = (size_t)p.T * (size_t)p.N * sizeof(float);
+  int S = router_k_splits(p);
+  if ((size_t)S * plane > logits_bytes) S = (int)(logits_bytes / plane);
+  if (S < 1) return cudaErrorInvalidValue;
+  const int k_len = ((p.d + S - 1) / S + kLBK - 1) / kLBK * kLBK;
+  dim3 grid((unsigned)((p.N + kLBN - 1) / kLBN), (unsigned)((p.T + kLBT - 1) / kLBT), (unsigned)S);
   if (p.dtype == MOE_BF16)
     router_logits_kernel<__nv_bfloat16><<<grid, kLThreads, 0, s>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)W_r, p.T, p.N, p.d, logits);
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)W_r, p.T, p.N, p.d, k_len, logits);
   else
     router_logits_kernel<float><<<grid, kLThreads, 0, s>>>((const float*)x, (const float*)W_r, p.T,
-                                                           p.N, p.d, logits);
+                                                           p.N, p.d, k_len, logits);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
 
-  SelectArgs a{logits, b, p.T, p.N, p.k, p.G, p.TG, p.score_fn, p.group_score, p.normalize,
+  SelectArgs a{logits, S, b, p.T, p.N, p.k, p.G, p.TG, p.score_fn, p.group_score, p.normalize,
                p.route_scale, idx, gates};
   const int warps = 8;
   unsigned blocks = (unsigned)((p.T + warps - 1) / warps);
