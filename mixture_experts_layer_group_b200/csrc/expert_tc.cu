@@ -27,13 +27,15 @@
 // CTA roles (192 threads, one CTA per SM, persistent):
 //   warp 0      scheduler + TMA producer (one lane): takes a unit id, hands it
 //               to the other roles through a shared-memory ring, then loads
-//               A 2 x 128 x 64 and B <= 256 x 64 bf16 per stage into a 3-stage
-//               ring of 64 KB; weights read by one unit only are evict-first
+//               A 2 x 128 x 64 and B <= 256 x 64 bf16 per stage. Stages are
+//               variable-size pieces (32 KB + 4 KB per 32 tokens) of a 204 KB
+//               byte ring, so units with few tokens keep more weight bytes in
+//               flight; weights read by one unit only are evict-first
 //   warp 1      TMEM owner + UMMA issuer (one lane): 2 x 4 x (128 x N x 16)
 //               per stage. TMEM holds two buffers of 2 x 128 fp32 columns: a
 //               unit of <= 128 tokens takes one buffer (the next unit's MMAs
 //               overlap its epilogue), a larger unit takes both (2 x 256)
-//   warps 2..13 epilogue, three warps per TMEM lane quadrant taking turns on
+//   warps 2..9  epilogue, two warps per TMEM lane quadrant taking turns on
 //               32-token blocks: each warp reads its quadrant, applies SwiGLU
 //               or the gate, transposes the 32 x 32 block through its own
 //               shared-memory tile (bf16) and writes 64-byte token-row
@@ -49,24 +51,26 @@
 namespace moe {
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kSlots = 8;                         // stages in flight at most
 constexpr int kBK = 64;                           // bf16 per K chunk: one 128 B swizzle row
 constexpr int kMaxTok = kTcBM;                    // tokens per unit (<= 256)
 constexpr int kTokBox = 32;                       // token rows per TMA box
+constexpr int kBoxBytes = kTokBox * kBK * 2;      // 4 KB
 constexpr int kHalfBytes = 128 * kBK * 2;         // 16 KB: one M = 128 weight tile
 constexpr int kATileBytes = 2 * kHalfBytes;       // 32 KB: two of them
-constexpr int kBTileBytes = kMaxTok * kBK * 2;    // 32 KB
-constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kMaxStageBytes = kATileBytes + (kMaxTok / kTokBox) * kBoxBytes;  // 64 KB
+constexpr int kRingBytes = 51 * 4096;             // 204 KB of variable-size stages
 constexpr int kBufCols = 256;                     // fp32 columns per accumulator buffer
 constexpr int kTmemCols = 2 * kBufCols;           // 2 buffers
-constexpr int kEpiWarps = 12;                     // three per TMEM lane quadrant
+constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kRing = 8;                          // unit ids in flight between the roles
 constexpr int kTPitch = 40;                       // bf16 per row of a warp's 32 x 32 tile (80 B)
 constexpr int kTBytes = kEpiWarps * 32 * kTPitch * 2;  // one tile per epilogue warp
 constexpr int kBarrierBytes = 512;
-constexpr int kSmemBytes = kStages * kStageBytes + kTBytes + 1024 + kBarrierBytes;
+constexpr int kSmemBytes = kRingBytes + kTBytes + 1024 + kBarrierBytes;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kMaxStageBytes * 3 <= kRingBytes, "ring holds three full stages");
 static_assert(kEpiWarps % 4 == 0, "whole quadrants");
 static_assert(kMaxTok <= kBufCols && kMaxTok % kTokBox == 0, "token chunk");
 
@@ -163,8 +167,9 @@ struct AccPlan {
 };
 
 struct Shared {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kSlots];
+  uint64_t empty[kSlots];
+  uint32_t slot_off[kSlots];  // byte offset of each stage in the ring
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t ring_full[kRing];
@@ -201,15 +206,15 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* tiles = reinterpret_cast<float*>(smem + kStages * kStageBytes);
-  Shared& sh = *reinterpret_cast<Shared*>(smem + kStages * kStageBytes + kTBytes);
+  float* tiles = reinterpret_cast<float*>(smem + kRingBytes);
+  Shared& sh = *reinterpret_cast<Shared*>(smem + kRingBytes + kTBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int total_units = __ldg(p.unit_base + p.N + 1);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSlots; ++s) {
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], 1);
     }
@@ -249,6 +254,40 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
       // tiles shared by the chunks of a large group stay at normal priority
       const uint64_t pol_once = policy_evict_first();
       const uint64_t pol_shared = policy_evict_normal();
+      // Ring allocation. Stages are placed back to back in fill order and
+      // freed in the same order by the MMA issuer's commits, so the bytes in
+      // use form one circular interval [offset of the oldest unfreed fill,
+      // head). A stage that does not fit before the end restarts at 0.
+      uint32_t off_of[kSlots];
+      uint32_t head = 0, oldest = 0;
+      auto acquire = [&](uint32_t j, uint32_t sz, uint32_t& pos) -> bool {
+        for (;;) {
+          const uint32_t inflight = j - oldest;
+          bool fits = false;
+          if (inflight == 0) {
+            pos = head + sz <= (uint32_t)kRingBytes ? head : 0u;
+            fits = true;
+          } else if (inflight < (uint32_t)kSlots) {
+            const uint32_t tail = off_of[oldest % kSlots];
+            if (tail < head) {  // in use: [tail, head)
+              if (head + sz <= (uint32_t)kRingBytes) {
+                pos = head;
+                fits = true;
+              } else if (sz <= tail) {
+                pos = 0;
+                fits = true;
+              }
+            } else if (head + sz <= tail) {  // in use wraps: [tail, end) + [0, head)
+              pos = head;
+              fits = true;
+            }
+          }
+          if (fits) return true;
+          // wait for the oldest fill to be consumed
+          if (!mbar_wait_bounded(&sh.empty[oldest % kSlots], (oldest / kSlots) & 1u, abort_flag)) return false;
+          ++oldest;
+        }
+      };
       bool ok = true;
       for (int i = 0;; ++i) {
         const int q = i % kRing;
@@ -266,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         const int K = shared ? p.k_shared : p.k_routed;
         const int nk = (K + kBK - 1) / kBK;
         const int nbox = (un.ntok + kTokBox - 1) / kTokBox;
-        const uint32_t tx = kATileBytes + nbox * (kTokBox * kBK * 2);
+        const uint32_t tx = kATileBytes + nbox * kBoxBytes;
         const int rowA = (shared ? 0 : un.g * p.a_rows_per_expert) + un.f * p.tile_cols;
         const int rowB = __ldg(p.grp_row0 + un.g) + un.tok0;
         const CUtensorMap* ta0 = shared ? &p.a0_shared : &p.a0_routed;
@@ -278,18 +317,22 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         MOE_TRACE_VAL(MODE, i, 7, (unsigned long long)un.ntok | ((unsigned long long)un.tok0 << 16) |
                                       ((unsigned long long)un.g << 32) | ((unsigned long long)un.f << 48));
         for (int kc = 0; kc < nk; ++kc, ++fills) {
-          const uint32_t s = fills % kStages, ph = (fills / kStages) & 1u;
-          if (!mbar_wait_bounded(&sh.empty[s], ph ^ 1u, abort_flag)) {
+          const uint32_t s = fills % kSlots;
+          uint32_t pos = 0;
+          if (!acquire(fills, tx, pos)) {
             ok = false;
             break;
           }
-          uint8_t* a_dst = smem + s * kStageBytes;
+          off_of[s] = pos;
+          head = pos + tx;
+          sh.slot_off[s] = pos;
+          uint8_t* a_dst = smem + pos;
           uint8_t* b_dst = a_dst + kATileBytes;
           mbar_arrive_expect_tx(&sh.full[s], tx);
           tma_load_2d_hint(a_dst, ta0, &sh.full[s], kc * kBK, rowA, pol);
           tma_load_2d_hint(a_dst + kHalfBytes, ta1, &sh.full[s], kc * kBK, rowA1, pol);
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d(b_dst + b * (kTokBox * kBK * 2), tb, &sh.full[s], kc * kBK, rowB + b * kTokBox);
+            tma_load_2d(b_dst + b * kBoxBytes, tb, &sh.full[s], kc * kBK, rowB + b * kTokBox);
         }
         MOE_TRACE(MODE, i, 1);
         if (!ok) break;
@@ -334,14 +377,14 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         tc_fence_after();
         const uint32_t d0 = tmem_base + base, d1 = tmem_base + base + stride;
         for (int kc = 0; kc < nk; ++kc) {
-          const uint32_t s = consumed % kStages, ph = (consumed / kStages) & 1u;
+          const uint32_t s = consumed % kSlots, ph = (consumed / kSlots) & 1u;
           if (!mbar_wait_bounded(&sh.full[s], ph, abort_flag)) {
             ok = false;
             break;
           }
           ++consumed;
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+          const uint32_t a_addr = smem_u32(smem + *reinterpret_cast<volatile uint32_t*>(&sh.slot_off[s]));
           const uint32_t b_addr = a_addr + kATileBytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
@@ -475,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
   if (warp == 0 && lane == 0) {
     // wait for any stage fill that was issued but never observed complete
     for (uint32_t j = sh.consumed; j < fills; ++j) {
-      const uint32_t s = j % kStages, ph = (j / kStages) & 1u;
+      const uint32_t s = j % kSlots, ph = (j / kSlots) & 1u;
       int dummy = 0;
       if (!mbar_wait_bounded(&sh.full[s], ph, &dummy)) {
         set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
