@@ -135,6 +135,28 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def rank_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 without it)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def token_shape_for_rank(s: mi.LayerShape, rank: int) -> mi.LayerShape:
+    """Every rank holds the same weights; its token batch comes from its own seed."""
+    return s.with_(seed=(s.seed + 17 * rank) & 0xFF)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def algorithmic(s: mi.LayerShape, counts: np.ndarray):
     """FLOPs and HBM bytes the layer must move (touched expert weights, router
     weights, x read, y written), and the SwiGLU GEMM's own bytes."""
@@ -165,7 +187,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     s = mi.SHAPES[args.config]
     # weights are the same replica everywhere; each rank draws its own token batch
-    sx = s.with_(seed=(s.seed + 17 * rank) & 0xFF)
+    sx = token_shape_for_rank(s, rank)
     w = mdev.device_all(s)
     x = mdev.device_tensor(sx, "x")
     cfg = moe.make_cfg(s.d, s.d_ff, s.n_routed, s.n_shared, s.top_k, s.n_groups, s.topk_groups, s.score,
@@ -232,10 +254,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms, stage_ms["gemm_swiglu"]], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms, _ = t.tolist()
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device="cuda")
     if rank != 0:
         return None
 
@@ -356,9 +375,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local_rank = rank_env()
     if args.impl == "reference":
         out = run_reference(args, rank, world)
         if out:
