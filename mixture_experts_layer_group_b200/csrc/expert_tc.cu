@@ -1,18 +1,22 @@
 // Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM,
-// operands staged by TMA), in "weights as M" orientation: every UMMA takes
-// 128 weight rows as its A operand (M = 128) and the group's token rows as B
-// (N = the tokens of the unit rounded up to 16, at most 256), so the MMA work
-// follows the real number of tokens per expert instead of a padded row tile.
-// A unit issues two such UMMAs per K step on one shared token tile (256
-// weight rows per unit). Two launches per layer:
+// operands staged by TMA), run by CTA pairs (clusters of 2) with pair UMMAs
+// (cta_group::2) in "weights as M" orientation. Every pair MMA takes 256
+// weight rows as its A operand (128 in each CTA's shared memory, M = 256)
+// and the group's token rows as B (N = the tokens of the unit rounded up to
+// 16, at most 256, half of them in each CTA), so each SM streams its own
+// weight rows but only half of the token rows, and the MMA work follows the
+// real number of tokens per expert instead of a padded row tile. A unit
+// issues two pair MMAs per K step on one shared token tile. Two launches per
+// layer:
 //
-//   SwiGLU GEMM  unit = (group, 128 features, <= 256 tokens): half 0 is 128
-//                rows of W1, half 1 the same 128 rows of W3, so TMEM lane i
-//                holds g and u of feature i for every token column; epilogue
+//   SwiGLU GEMM  unit = (group, 256 features, <= 256 tokens): CTA r holds
+//                features 128 r .. 128 r + 127 of the unit; half 0 of its
+//                rows is W1, half 1 the same rows of W3, so TMEM lane i holds
+//                g and u of one feature for every token column; epilogue
 //                h = silu(g) * u -> bf16
 //                ("Routed expert:" / "Shared expert:" steps g = x W1,
 //                u = x W3, a = g sigma(g), h = a (.) u)
-//   gate GEMM    unit = (group, 256 model columns, <= 256 tokens):
+//   gate GEMM    unit = (group, 512 model columns, <= 256 tokens):
 //                E^T = W2 h^T; epilogue E * G (the token slot's gate; 1 for
 //                the shared MLP) -> bf16 row of the slot
 //                ("E_i = h W2", "y_routed = sum G_i E_i")
@@ -20,27 +24,29 @@
 // Groups 0..N-1 are the routed experts over their expert-contiguous token
 // rows; group N is the fused shared MLP over all T tokens, in the same
 // persistent launch. Units of one group are consecutive, weight-tile major
-// and token-chunk minor. CTAs take units from a global counter, so the
-// chunks that share a weight tile start together (they read it once through
-// L2) and the last units balance across SMs.
+// and token-chunk minor. The pair's first CTA takes units from a global
+// counter, so the chunks that share a weight tile start together (they read
+// it once through L2) and the last units balance across SMs.
 //
-// CTA roles (192 threads, one CTA per SM, persistent):
-//   warp 0      scheduler + TMA producer (one lane): takes a unit id, hands it
-//               to the other roles through a shared-memory ring, then loads
-//               A 2 x 128 x 64 and B <= 256 x 64 bf16 per stage. Stages are
-//               variable-size pieces (32 KB + 4 KB per 32 tokens) of a 204 KB
-//               byte ring, so units with few tokens keep more weight bytes in
-//               flight; weights read by one unit only are evict-first
-//   warp 1      TMEM owner + UMMA issuer (one lane): 2 x 4 x (128 x N x 16)
-//               per stage. TMEM holds two buffers of 2 x 128 fp32 columns: a
-//               unit of <= 128 tokens takes one buffer (the next unit's MMAs
+// CTA roles (320 threads, one CTA per SM, persistent; the same roles in both
+// CTAs of a pair except the MMA issuer, which only the first CTA has):
+//   warp 0      TMA producer (one lane). In CTA 0 it also takes unit ids and
+//               hands them to both CTAs through shared-memory rings. Stages
+//               are variable-size pieces (32 KB of weights + 4 KB per 32 token
+//               rows) of a 204 KB byte ring; the bytes of both CTAs complete
+//               on CTA 0's stage barrier; weights read by one unit only are
+//               evict-first
+//   warp 1      TMEM owner (both CTAs, pair allocation) + UMMA issuer (CTA 0,
+//               one lane): 2 x 4 pair MMAs (256 x N x 16) per stage. Each
+//               CTA's TMEM holds two buffers of 2 x 128 fp32 columns: a unit
+//               of <= 128 tokens takes one buffer (the next unit's MMAs
 //               overlap its epilogue), a larger unit takes both (2 x 256)
 //   warps 2..9  epilogue, two warps per TMEM lane quadrant taking turns on
 //               32-token blocks: each warp reads its quadrant, applies SwiGLU
 //               or the gate, transposes the 32 x 32 block through its own
 //               shared-memory tile (bf16) and writes 64-byte token-row
 //               segments; no barrier between epilogue warps per block
-// Every mbarrier wait is bounded; on a timeout the CTA records
+// Every mbarrier wait is bounded; on a timeout a CTA records
 // MOE_DEV_WAIT_TIMEOUT, drains its own copies and MMAs (bounded again),
 // frees its tensor memory and exits.
 #include <cuda.h>
@@ -56,9 +62,9 @@ constexpr int kBK = 64;                           // bf16 per K chunk: one 128 B
 constexpr int kMaxTok = kTcBM;                    // tokens per unit (<= 256)
 constexpr int kTokBox = 32;                       // token rows per TMA box
 constexpr int kBoxBytes = kTokBox * kBK * 2;      // 4 KB
-constexpr int kHalfBytes = 128 * kBK * 2;         // 16 KB: one M = 128 weight tile
-constexpr int kATileBytes = 2 * kHalfBytes;       // 32 KB: two of them
-constexpr int kMaxStageBytes = kATileBytes + (kMaxTok / kTokBox) * kBoxBytes;  // 64 KB
+constexpr int kHalfBytes = 128 * kBK * 2;         // 16 KB: 128 weight rows of one half
+constexpr int kATileBytes = 2 * kHalfBytes;       // 32 KB: this CTA's rows of both halves
+constexpr int kMaxStageBytes = kATileBytes + (kMaxTok / 2 / kTokBox) * kBoxBytes;  // 48 KB
 constexpr int kRingBytes = 51 * 4096;             // 204 KB of variable-size stages
 constexpr int kBufCols = 256;                     // fp32 columns per accumulator buffer
 constexpr int kTmemCols = 2 * kBufCols;           // 2 buffers
@@ -72,7 +78,7 @@ constexpr int kSmemBytes = kRingBytes + kTBytes + 1024 + kBarrierBytes;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kMaxStageBytes * 3 <= kRingBytes, "ring holds three full stages");
 static_assert(kEpiWarps % 4 == 0, "whole quadrants");
-static_assert(kMaxTok <= kBufCols && kMaxTok % kTokBox == 0, "token chunk");
+static_assert(kMaxTok <= kBufCols && kMaxTok % (2 * kTokBox) == 0, "token chunk");
 
 enum Mode : int { kSwiGLU = 0, kGateDown = 1 };
 
@@ -109,7 +115,7 @@ struct TcParams {
   int k_routed, k_shared;        // reduction length (d | F, d | nsF)
   int cols_routed, cols_shared;  // output columns (F, nsF | d, d)
   int a_rows_per_expert;         // rows of the stacked weight tensor per routed expert (F | d)
-  int tile_cols;                 // output columns per unit (128 | 256)
+  int tile_cols;                 // output columns per unit (256 | 512)
   __nv_bfloat16* out_routed;
   int64_t ld_routed;
   __nv_bfloat16* out_shared;
@@ -146,10 +152,11 @@ MOE_DEV Unit decode_unit(const TcParams& p, int u) {
   return un;
 }
 
-// Accumulator placement. A unit of <= 128 tokens takes one buffer (its two
-// halves at columns base and base + 128); a larger unit takes both buffers
-// (halves at columns 0 and 256). The MMA issuer and every epilogue thread
-// replay the same sequence, so they agree on every placement.
+// Accumulator placement (identical in both CTAs). A unit of <= 128 tokens
+// takes one buffer (its two halves at columns base and base + 128); a larger
+// unit takes both buffers (halves at columns 0 and 256). The MMA issuer and
+// every epilogue thread replay the same sequence, so they agree on every
+// placement.
 struct AccPlan {
   uint32_t next = 0;
   MOE_DEV void place(int ntok, uint32_t& mask, uint32_t& base, uint32_t& stride) const {
@@ -167,19 +174,19 @@ struct AccPlan {
 };
 
 struct Shared {
-  uint64_t full[kSlots];
-  uint64_t empty[kSlots];
-  uint32_t slot_off[kSlots];  // byte offset of each stage in the ring
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
-  uint64_t ring_full[kRing];
-  uint64_t ring_empty[kRing];
-  uint64_t drained;
+  uint64_t full[kSlots];       // CTA 0: stage bytes of both CTAs landed
+  uint64_t empty[kSlots];      // both: the pair MMAs finished reading the stage
+  uint64_t acc_full[2];        // both: accumulator buffer complete
+  uint64_t acc_empty[2];       // CTA 0: both CTAs' epilogues released the buffer
+  uint64_t ring_full[kRing];   // both: unit id published
+  uint64_t ring_empty[kRing];  // CTA 0: every reader of the pair took the id
+  uint64_t drained;            // both: all pair MMAs completed
+  uint32_t slot_off[kSlots];   // byte offset of each stage in the ring
   int ring[kRing];
-  int epi_unit[2];    // the epilogue leader's unit for the 4 epilogue warps
+  int epi_unit[2];             // the epilogue leader's unit for the epilogue warps
   uint32_t tmem_base;
   int abort_flag;
-  uint32_t consumed;  // stage fills the MMA issuer observed complete
+  uint32_t consumed;           // stage fills the MMA issuer observed complete
 };
 
 // Barrier among the epilogue warps only (id 1; id 0 is __syncthreads).
@@ -211,7 +218,12 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the pair MMAs and takes the units
+  const bool first = rank == 0;
   const int total_units = __ldg(p.unit_base + p.N + 1);
+  // this CTA's rows of each 256-row weight half, and the offset between halves
+  const int rank_rows = 128 * (int)rank;
+  const int half_rows = MODE == kSwiGLU ? 0 : 256;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
@@ -220,11 +232,11 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.acc_full[b], 1);
-      mbar_init(&sh.acc_empty[b], kEpiWarps);
+      mbar_init(&sh.acc_empty[b], 2 * kEpiWarps);
     }
     for (int q = 0; q < kRing; ++q) {
       mbar_init(&sh.ring_full[q], 1);
-      mbar_init(&sh.ring_empty[q], 2);  // MMA issuer + epilogue leader
+      mbar_init(&sh.ring_empty[q], 4);  // both CTAs: producer or MMA issuer, epilogue leader
     }
     mbar_init(&sh.drained, 1);
     sh.abort_flag = 0;
@@ -237,14 +249,16 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
     if (MODE == kSwiGLU) tma_prefetch_desc(&p.a1_routed);
   }
   if (warp == 1) {
-    tmem_alloc(&sh.tmem_base, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(&sh.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers and tensor memory of both CTAs are ready
   tc_fence_after();
   const uint32_t tmem_base = sh.tmem_base;
   volatile int* abort_flag = &sh.abort_flag;
+  auto peer = [&](const void* local) { return map_to_rank(smem_u32(local), rank ^ 1u); };
+  auto in_first = [&](const void* local) { return map_to_rank(smem_u32(local), 0u); };
 
   uint32_t fills = 0;  // producer: stage fills issued
   if (warp == 0) {
@@ -254,10 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
       // tiles shared by the chunks of a large group stay at normal priority
       const uint64_t pol_once = policy_evict_first();
       const uint64_t pol_shared = policy_evict_normal();
-      // Ring allocation. Stages are placed back to back in fill order and
-      // freed in the same order by the MMA issuer's commits, so the bytes in
-      // use form one circular interval [offset of the oldest unfreed fill,
-      // head). A stage that does not fit before the end restarts at 0.
+      // Ring allocation (identical in both CTAs, so stage offsets match).
+      // Stages are placed back to back in fill order and freed in the same
+      // order by the pair MMAs' commits, so the bytes in use form one circular
+      // interval [offset of the oldest unfreed fill, head). A stage that does
+      // not fit before the end restarts at 0.
       uint32_t off_of[kSlots];
       uint32_t head = 0, oldest = 0;
       auto acquire = [&](uint32_t j, uint32_t sz, uint32_t& pos) -> bool {
@@ -284,33 +299,46 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           }
           if (fits) return true;
           // wait for the oldest fill to be consumed
-          if (!mbar_wait_bounded(&sh.empty[oldest % kSlots], (oldest / kSlots) & 1u, abort_flag)) return false;
+          if (!mbar_wait_cluster_bounded(&sh.empty[oldest % kSlots], (oldest / kSlots) & 1u, abort_flag))
+            return false;
           ++oldest;
         }
       };
       bool ok = true;
       for (int i = 0;; ++i) {
         const int q = i % kRing;
-        if (!mbar_wait_bounded(&sh.ring_empty[q], ((i / kRing) & 1) ^ 1, abort_flag)) {
-          ok = false;
-          break;
+        int u;
+        if (first) {
+          if (!mbar_wait_cluster_bounded(&sh.ring_empty[q], ((i / kRing) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          u = atomicAdd(p.sched, 1);
+          if (u >= total_units) u = -1;
+          sh.ring[q] = u;
+          st_cluster_u32(peer(&sh.ring[q]), (uint32_t)u);
+          mbar_arrive(&sh.ring_full[q]);
+          mbar_arrive_cluster(peer(&sh.ring_full[q]));
+        } else {
+          if (!mbar_wait_cluster_bounded(&sh.ring_full[q], (i / kRing) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          u = load_volatile(&sh.ring[q]);
+          mbar_arrive_cluster(in_first(&sh.ring_empty[q]));
         }
-        int u = atomicAdd(p.sched, 1);
-        if (u >= total_units) u = -1;
-        sh.ring[q] = u;
-        mbar_arrive(&sh.ring_full[q]);
         if (u < 0) break;
         const Unit un = decode_unit(p, u);
         const bool shared = un.g == p.N;
         const int K = shared ? p.k_shared : p.k_routed;
         const int nk = (K + kBK - 1) / kBK;
-        const int nbox = (un.ntok + kTokBox - 1) / kTokBox;
+        const int half_n = ((un.ntok + 15) & ~15) / 2;  // token rows per CTA
+        const int nbox = (half_n + kTokBox - 1) / kTokBox;
         const uint32_t tx = kATileBytes + nbox * kBoxBytes;
-        const int rowA = (shared ? 0 : un.g * p.a_rows_per_expert) + un.f * p.tile_cols;
-        const int rowB = __ldg(p.grp_row0 + un.g) + un.tok0;
+        const int rowA = (shared ? 0 : un.g * p.a_rows_per_expert) + un.f * p.tile_cols + rank_rows;
+        const int rowB = __ldg(p.grp_row0 + un.g) + un.tok0 + (int)rank * half_n;
         const CUtensorMap* ta0 = shared ? &p.a0_shared : &p.a0_routed;
         const CUtensorMap* ta1 = MODE == kSwiGLU ? (shared ? &p.a1_shared : &p.a1_routed) : ta0;
-        const int rowA1 = MODE == kSwiGLU ? rowA : rowA + 128;  // W3 rows | next 128 W2 rows
         const CUtensorMap* tb = shared ? &p.b_shared : &p.b_routed;
         const uint64_t pol = un.nchunks == 1 ? pol_once : pol_shared;
         MOE_TRACE(MODE, i, 0);
@@ -328,11 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           sh.slot_off[s] = pos;
           uint8_t* a_dst = smem + pos;
           uint8_t* b_dst = a_dst + kATileBytes;
-          mbar_arrive_expect_tx(&sh.full[s], tx);
-          tma_load_2d_hint(a_dst, ta0, &sh.full[s], kc * kBK, rowA, pol);
-          tma_load_2d_hint(a_dst + kHalfBytes, ta1, &sh.full[s], kc * kBK, rowA1, pol);
+          const uint32_t full_bar = in_first(&sh.full[s]);
+          if (first) mbar_arrive_expect_tx(&sh.full[s], 2 * tx);  // this CTA's bytes and the peer's
+          tma_load_2d_pair(a_dst, ta0, full_bar, kc * kBK, rowA, pol);
+          tma_load_2d_pair(a_dst + kHalfBytes, ta1, full_bar, kc * kBK, rowA + half_rows, pol);
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d(b_dst + b * kBoxBytes, tb, &sh.full[s], kc * kBK, rowB + b * kTokBox);
+            tma_load_2d_pair(b_dst + b * kBoxBytes, tb, full_bar, kc * kBK, rowB + b * kTokBox, pol_shared);
         }
         MOE_TRACE(MODE, i, 1);
         if (!ok) break;
@@ -344,15 +373,15 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer --
-    if (lane == 0) {
+    // ------------------------------------------------- MMA issuer (CTA 0) --
+    if (lane == 0 && first) {
       uint32_t consumed = 0;
       uint32_t uses[2] = {0u, 0u};
       AccPlan plan;
       bool ok = true;
       for (int i = 0; ok; ++i) {
         const int q = i % kRing;
-        if (!mbar_wait_bounded(&sh.ring_full[q], (i / kRing) & 1, abort_flag)) {
+        if (!mbar_wait_cluster_bounded(&sh.ring_full[q], (i / kRing) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -362,14 +391,14 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         const Unit un = decode_unit(p, u);
         const int K = un.g == p.N ? p.k_shared : p.k_routed;
         const int nk = (K + kBK - 1) / kBK;
-        const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)((un.ntok + 15) & ~15));
+        const uint32_t idesc = idesc_bf16_f32(256, (uint32_t)((un.ntok + 15) & ~15));
         uint32_t mask, base, stride;
         plan.place(un.ntok, mask, base, stride);
         plan.advance(un.ntok);
         MOE_TRACE(MODE, i, 2);
         for (int b = 0; b < 2 && ok; ++b)
           if ((mask >> b) & 1u) {
-            ok = mbar_wait_bounded(&sh.acc_empty[b], (uses[b] & 1u) ^ 1u, abort_flag);
+            ok = mbar_wait_cluster_bounded(&sh.acc_empty[b], (uses[b] & 1u) ^ 1u, abort_flag);
             ++uses[b];
           }
         if (!ok) break;
@@ -378,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         const uint32_t d0 = tmem_base + base, d1 = tmem_base + base + stride;
         for (int kc = 0; kc < nk; ++kc) {
           const uint32_t s = consumed % kSlots, ph = (consumed / kSlots) & 1u;
-          if (!mbar_wait_bounded(&sh.full[s], ph, abort_flag)) {
+          if (!mbar_wait_cluster_bounded(&sh.full[s], ph, abort_flag)) {
             ok = false;
             break;
           }
@@ -389,14 +418,18 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32);
-            umma_bf16(d0, smem_desc_sw128(a_addr + kk * 32), bdesc, idesc, (kc | kk) != 0);
-            umma_bf16(d1, smem_desc_sw128(a_addr + kHalfBytes + kk * 32), bdesc, idesc, (kc | kk) != 0);
+            umma_bf16_pair(d0, smem_desc_sw128(a_addr + kk * 32), bdesc, idesc, (kc | kk) != 0);
+            umma_bf16_pair(d1, smem_desc_sw128(a_addr + kHalfBytes + kk * 32), bdesc, idesc, (kc | kk) != 0);
           }
-          umma_commit(&sh.empty[s]);
+          umma_commit_pair(smem_u32(&sh.empty[s]));
+          umma_commit_pair(peer(&sh.empty[s]));
         }
         if (ok) {
-          if (mask & 1u) umma_commit(&sh.acc_full[0]);
-          if (mask & 2u) umma_commit(&sh.acc_full[1]);
+          for (int b = 0; b < 2; ++b)
+            if ((mask >> b) & 1u) {
+              umma_commit_pair(smem_u32(&sh.acc_full[b]));
+              umma_commit_pair(peer(&sh.acc_full[b]));
+            }
         }
         MOE_TRACE(MODE, i, 4);
       }
@@ -404,11 +437,14 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         *abort_flag = 1;
         set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
       }
-      // all MMAs issued by this thread have completed once `drained` fires
-      umma_commit(&sh.drained);
-      int no_abort = 0;  // wait for the MMAs even when unwinding
-      if (!mbar_wait_bounded(&sh.drained, 0, &no_abort)) set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
+      // all pair MMAs have completed once `drained` fires (in both CTAs)
+      umma_commit_pair(smem_u32(&sh.drained));
+      umma_commit_pair(peer(&sh.drained));
       sh.consumed = consumed;
+    }
+    if (lane == 0) {
+      int no_abort = 0;  // wait for the MMAs even when unwinding
+      if (!mbar_wait_cluster_bounded(&sh.drained, 0, &no_abort)) set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
     }
     __syncwarp();
   } else {
@@ -426,16 +462,17 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
       if (leader) {
         int u = -2;
         const int qr = i % kRing;
-        if (mbar_wait_bounded(&sh.ring_full[qr], (i / kRing) & 1, abort_flag)) {
+        if (mbar_wait_cluster_bounded(&sh.ring_full[qr], (i / kRing) & 1, abort_flag)) {
           u = load_volatile(&sh.ring[qr]);
-          mbar_arrive(&sh.ring_empty[qr]);
+          if (first) mbar_arrive(&sh.ring_empty[qr]);
+          else mbar_arrive_cluster(in_first(&sh.ring_empty[qr]));
           if (u >= 0) {
             const Unit un = decode_unit(p, u);
             uint32_t mask, base, stride;
             plan.place(un.ntok, mask, base, stride);
             bool ok = true;
             for (int b = 0; b < 2 && ok; ++b)
-              if ((mask >> b) & 1u) ok = mbar_wait_bounded(&sh.acc_full[b], uses[b] & 1u, abort_flag);
+              if ((mask >> b) & 1u) ok = mbar_wait_cluster_bounded(&sh.acc_full[b], uses[b] & 1u, abort_flag);
             if (!ok) u = -2;
           }
         }
@@ -466,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
 #pragma unroll 1
       for (int hh = 0; hh < kHalves; ++hh) {
         // this warp's 32 output columns of the unit
-        const int c0 = un.f * p.tile_cols + (MODE == kSwiGLU ? 0 : 128 * hh) + 32 * q;
+        const int c0 = un.f * p.tile_cols + half_rows * hh + rank_rows + 32 * q;
 #pragma unroll 1
         for (int j0 = 32 * sub; j0 < un.ntok; j0 += 32 * (kEpiWarps / 4)) {
           const int tok = j0 + lane;
@@ -508,28 +545,33 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
       __syncwarp();
       if (leader) MOE_TRACE(MODE, i, 6);
       if (lane == 0) {
-        if (mask & 1u) mbar_arrive(&sh.acc_empty[0]);
-        if (mask & 2u) mbar_arrive(&sh.acc_empty[1]);
+        for (int b = 0; b < 2; ++b)
+          if ((mask >> b) & 1u) {
+            if (first) mbar_arrive(&sh.acc_empty[b]);
+            else mbar_arrive_cluster(in_first(&sh.acc_empty[b]));
+          }
       }
     }
   }
 
   __syncthreads();
-  if (warp == 0 && lane == 0) {
+  if (warp == 0 && lane == 0 && first) {
     // wait for any stage fill that was issued but never observed complete
+    // (its bytes from both CTAs land on this CTA's stage barrier)
     for (uint32_t j = sh.consumed; j < fills; ++j) {
       const uint32_t s = j % kSlots, ph = (j / kSlots) & 1u;
       int dummy = 0;
-      if (!mbar_wait_bounded(&sh.full[s], ph, &dummy)) {
+      if (!mbar_wait_cluster_bounded(&sh.full[s], ph, &dummy)) {
         set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
         break;
       }
     }
   }
-  __syncthreads();
+  tc_fence_before();
+  cluster_sync();  // neither CTA leaves while the other may still touch its shared memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
@@ -568,18 +610,37 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
 }
 
 template <int MODE>
-cudaError_t launch_one(const TcParams& prm, int grid, cudaStream_t s) {
+cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s) {
   static int configured_device = -1;
+  static int max_clusters = 0;
   int dev = 0;
   cudaGetDevice(&dev);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (configured_device != dev) {
     cudaError_t e = cudaFuncSetAttribute(expert_gemm_tc_kernel<MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, expert_gemm_tc_kernel<MODE>, &cfg);
+    if (e != cudaSuccess) return e;
+    max_clusters = n > 0 ? n : 1;
     configured_device = dev;
   }
-  expert_gemm_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(prm);
-  return cudaGetLastError();
+  int clusters = max_clusters;
+  if (max_units < clusters) clusters = max_units > 0 ? max_units : 1;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  return cudaLaunchKernelEx(&cfg, expert_gemm_tc_kernel<MODE>, prm);
 }
 
 }  // namespace
@@ -619,8 +680,7 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g1.status = a.status;
   const int64_t max_cols1 = p.F > p.nsF ? p.F : p.nsF;
   const int64_t units1 = chunks_bound * ((max_cols1 + kTcBN1 - 1) / kTcBN1);
-  const int grid1 = (int)(units1 < sms ? units1 : sms);
-  cudaError_t err = launch_one<kSwiGLU>(g1, grid1 > 0 ? grid1 : 1, s);
+  cudaError_t err = launch_one<kSwiGLU>(g1, (int)(units1 < sms ? units1 : sms), s);
   if (err == cudaSuccess && between) err = cudaEventRecord(between, s);
   if (err != cudaSuccess) return err;
 
@@ -648,8 +708,7 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g2.gate_perm = a.gate_perm;
   g2.status = a.status;
   const int64_t units2 = chunks_bound * ((p.d + kTcBN2 - 1) / kTcBN2);
-  const int grid2 = (int)(units2 < sms ? units2 : sms);
-  return launch_one<kGateDown>(g2, grid2 > 0 ? grid2 : 1, s);
+  return launch_one<kGateDown>(g2, (int)(units2 < sms ? units2 : sms), s);
 }
 
 }  // namespace moe

@@ -10,14 +10,14 @@
 
 namespace moe {
 
-// Tile sizes of the tensor-core grouped GEMMs: a unit covers at most
-// kTcBM token rows of one group (UMMA N) and kTcBN1 SwiGLU features (two
-// UMMAs of M = 128, each 64 W1 rows stacked over 64 W3 rows) or kTcBN2 model
-// columns of the down projection (two UMMAs of M = 128). The fp32 SIMT GEMMs
-// use 64 x 64 tiles.
+// Tile sizes of the tensor-core grouped GEMMs (run by CTA pairs): a unit
+// covers at most kTcBM token rows of one group (UMMA N) and kTcBN1 SwiGLU
+// features (two pair UMMAs of M = 256: W1 rows and the same W3 rows) or
+// kTcBN2 model columns of the down projection (two pair UMMAs of M = 256).
+// The fp32 SIMT GEMMs use 64 x 64 tiles.
 constexpr int kTcBM = 256;
-constexpr int kTcBN1 = 128;
-constexpr int kTcBN2 = 256;
+constexpr int kTcBN1 = 256;
+constexpr int kTcBN2 = 512;
 constexpr int kSimtBM = 64;
 constexpr int kSimtBN = 64;
 constexpr int kChunkTokens = 32;  // dispatch: tokens per warp chunk
