@@ -175,6 +175,24 @@ MOE_DEV void tma_load_2d_pair(void* smem_dst, const void* tmap, uint32_t bar_clu
       : "memory");
 }
 
+// 2-D tiled store of a shared-memory box to global memory (bulk group). The
+// box start (c0, c1) must be non-negative and c0 a multiple of 16 bytes'
+// worth of elements; rows/columns beyond the tensor are clipped.
+MOE_DEV void tma_store_2d(const void* tmap, const void* smem_src, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+MOE_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until at most N committed bulk groups still read their shared-memory source.
+template <int N>
+MOE_DEV void bulk_wait_group_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+// Waits until every committed bulk group has completed.
+MOE_DEV void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Orders this thread's generic shared-memory writes before later async-proxy reads.
+MOE_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 MOE_DEV uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -334,6 +352,16 @@ MOE_DEV uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 MOE_DEV float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
+
+// silu(g) = g sigma(g) with sigma(g) = (1 + tanh(g / 2)) / 2 from the
+// hardware tanh approximation (one special-function op; relative error of
+// sigma about 1e-3, below the bf16 rounding the result gets).
+MOE_DEV float silu_tanh(float g) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * g));
+  const float hg = 0.5f * g;
+  return fmaf(hg, t, hg);
+}
 
 MOE_DEV void set_status(unsigned* status, unsigned bits) {
   if (status) atomicOr(status, bits);

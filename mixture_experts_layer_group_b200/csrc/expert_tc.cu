@@ -44,8 +44,9 @@
 //   warps 2..9  epilogue, two warps per TMEM lane quadrant taking turns on
 //               32-token blocks: each warp reads its quadrant, applies SwiGLU
 //               or the gate, transposes the 32 x 32 block through its own
-//               shared-memory tile (bf16) and writes 64-byte token-row
-//               segments; no barrier between epilogue warps per block
+//               shared-memory tile (bf16) and writes it with
+//               one TMA tensor store (a ragged last block with 64-byte row
+//               stores); no barrier between epilogue warps per block
 // Every mbarrier wait is bounded; on a timeout a CTA records
 // MOE_DEV_WAIT_TIMEOUT, drains its own copies and MMAs (bounded again),
 // frees its tensor memory and exits.
@@ -65,14 +66,14 @@ constexpr int kBoxBytes = kTokBox * kBK * 2;      // 4 KB
 constexpr int kHalfBytes = 128 * kBK * 2;         // 16 KB: 128 weight rows of one half
 constexpr int kATileBytes = 2 * kHalfBytes;       // 32 KB: this CTA's rows of both halves
 constexpr int kMaxStageBytes = kATileBytes + (kMaxTok / 2 / kTokBox) * kBoxBytes;  // 48 KB
-constexpr int kRingBytes = 51 * 4096;             // 204 KB of variable-size stages
+constexpr int kRingBytes = 52 * 4096;             // 208 KB of variable-size stages
 constexpr int kBufCols = 256;                     // fp32 columns per accumulator buffer
 constexpr int kTmemCols = 2 * kBufCols;           // 2 buffers
 constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kRing = 8;                          // unit ids in flight between the roles
-constexpr int kTPitch = 40;                       // bf16 per row of a warp's 32 x 32 tile (80 B)
-constexpr int kTBytes = kEpiWarps * 32 * kTPitch * 2;  // one tile per epilogue warp
+constexpr int kTileBytes = 32 * 32 * 2;           // a warp's dense 32 x 32 bf16 tile (TMA store box)
+constexpr int kTBytes = kEpiWarps * kTileBytes;        // one tile per epilogue warp
 constexpr int kBarrierBytes = 512;
 constexpr int kSmemBytes = kRingBytes + kTBytes + 1024 + kBarrierBytes;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -86,7 +87,7 @@ enum Mode : int { kSwiGLU = 0, kGateDown = 1 };
 // only with -DMOE_UNIT_TRACE for pipeline studies; a no-op otherwise.
 #ifdef MOE_UNIT_TRACE
 constexpr int kTraceCtas = 160, kTraceUnits = 160;
-__device__ unsigned long long g_unit_trace[2][kTraceCtas][kTraceUnits][8];
+__device__ unsigned long long g_unit_trace[2][kTraceCtas][kTraceUnits][16];
 #define MOE_TRACE_VAL(mode, unit_i, slot, value)                                        \
   do {                                                                                 \
     if (blockIdx.x < kTraceCtas && (unit_i) < kTraceUnits)                             \
@@ -107,6 +108,8 @@ struct TcParams {
   CUtensorMap a1_shared;  // Ws3 [nsF, d]     | unused
   CUtensorMap b_routed;   // x_perm [R, d]    | h_perm [R, F]
   CUtensorMap b_shared;   // x [T, d]         | h_sh [T, nsF]
+  CUtensorMap o_routed;   // h_perm [R, F]    | y_rows [R + T, d]   (32 x 32 store box)
+  CUtensorMap o_shared;   // h_sh [T, nsF]    | y_rows [R + T, d]
   const int32_t* unit_base;  // [N + 2]: units before group g; [N + 1] = total
   const int32_t* grp_row0;   // [N + 1]
   const int32_t* grp_rows;   // [N + 1]
@@ -120,6 +123,7 @@ struct TcParams {
   int64_t ld_routed;
   __nv_bfloat16* out_shared;
   int64_t ld_shared;
+  int out_row0_shared;           // first row of the shared MLP's rows in o_shared (0 | R)
   const float* gate_perm;        // [R] (gate-down mode)
   unsigned* status;
 };
@@ -184,10 +188,12 @@ struct Shared {
   uint32_t slot_off[kSlots];   // byte offset of each stage in the ring
   int ring[kRing];
   int epi_unit[2];             // the epilogue leader's unit for the epilogue warps
+  int epi_info[2][5];          // its decoded (g, f, tok0, ntok) and first output row
   uint32_t tmem_base;
   int abort_flag;
   uint32_t consumed;           // stage fills the MMA issuer observed complete
 };
+static_assert(sizeof(Shared) <= kBarrierBytes, "barrier block");
 
 // Barrier among the epilogue warps only (id 1; id 0 is __syncthreads).
 MOE_DEV void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
@@ -452,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
     const int q = warp & 3;                  // TMEM lane quadrant this warp may access
     const int ew = warp - 2;                 // epilogue warp: its transpose tile
     const int sub = ew >> 2;                 // which of the quadrant's warps
-    __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(tiles) + ew * 32 * kTPitch;
+    __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(tiles) + ew * kTileBytes);
     const bool leader = threadIdx.x == 64;
     uint32_t uses[2] = {0u, 0u};
     AccPlan plan;
@@ -468,6 +474,11 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           else mbar_arrive_cluster(in_first(&sh.ring_empty[qr]));
           if (u >= 0) {
             const Unit un = decode_unit(p, u);
+            sh.epi_info[i & 1][0] = un.g;
+            sh.epi_info[i & 1][1] = un.f;
+            sh.epi_info[i & 1][2] = un.tok0;
+            sh.epi_info[i & 1][3] = un.ntok;
+            sh.epi_info[i & 1][4] = un.g == p.N ? un.tok0 : __ldg(p.grp_row0 + un.g) + un.tok0;
             uint32_t mask, base, stride;
             plan.place(un.ntok, mask, base, stride);
             bool ok = true;
@@ -485,7 +496,11 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
       epi_sync();
       const int u = load_volatile(&sh.epi_unit[i & 1]);
       if (u < 0) break;
-      const Unit un = decode_unit(p, u);
+      Unit un;
+      un.g = load_volatile(&sh.epi_info[i & 1][0]);
+      un.f = load_volatile(&sh.epi_info[i & 1][1]);
+      un.tok0 = load_volatile(&sh.epi_info[i & 1][2]);
+      un.ntok = load_volatile(&sh.epi_info[i & 1][3]);
       uint32_t mask, base, stride;
       plan.place(un.ntok, mask, base, stride);
       plan.advance(un.ntok);
@@ -494,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
       if (leader) MOE_TRACE(MODE, i, 5);
       tc_fence_after();
       const bool shared = un.g == p.N;
-      const int64_t row_base = shared ? (int64_t)un.tok0 : (int64_t)__ldg(p.grp_row0 + un.g) + un.tok0;
+      const int64_t row_base = load_volatile(&sh.epi_info[i & 1][4]);
       __nv_bfloat16* out_base = shared ? p.out_shared : p.out_routed;
       const int64_t ld = shared ? p.ld_shared : p.ld_routed;
       const int cols = shared ? p.cols_shared : p.cols_routed;
@@ -511,6 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           // gate of this lane's token, spread to the column-owning lanes below
           float my_gate = 1.0f;
           if (MODE == kGateDown && !shared && tok < un.ntok) my_gate = __ldg(p.gate_perm + row);
+          if (leader && hh == 0 && j0 == 0) MOE_TRACE(MODE, i, 12);
           float v[32];
           {
             uint32_t a[32];
@@ -522,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
                 const float g = __uint_as_float(a[j]);
-                v[j] = __fdividef(g, 1.0f + __expf(-g)) * __uint_as_float(b[j]);
+                v[j] = silu_tanh(g) * __uint_as_float(b[j]);
               }
             } else {
               tmem_wait_ld();
@@ -530,15 +546,34 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
               for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]) * __shfl_sync(0xffffffffu, my_gate, j);
             }
           }
-          // transpose through this warp's tile: lane = column -> lane = token
-#pragma unroll
-          for (int j = 0; j < 32; ++j) tile[j * kTPitch + lane] = __float2bfloat16_rn(v[j]);
+          const bool probe = leader && hh == 0 && j0 == 0;
+          if (probe) MOE_TRACE(MODE, i, 8);
+          // transpose through this warp's tile: lane = column -> row = token
+          if (lane == 0) bulk_wait_group_read<0>();  // the previous block's store has read the tile
           __syncwarp();
-          uint4 rowv[4];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) rowv[c] = *reinterpret_cast<const uint4*>(tile + lane * kTPitch + 8 * c);
-          __syncwarp();
-          if (tok < un.ntok) store_row32(out_base + row * ld + c0, cols - c0, rowv);
+          for (int j = 0; j < 32; ++j) tile[j * 32 + lane] = __float2bfloat16_rn(v[j]);
+          const bool full_block = j0 + 32 <= un.ntok && c0 + 32 <= cols;
+          if (full_block) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (probe) MOE_TRACE(MODE, i, 9);
+            if (probe) MOE_TRACE(MODE, i, 10);
+            if (lane == 0) {
+              tma_store_2d(shared ? &p.o_shared : &p.o_routed, tile, c0,
+                           (int)(row_base + j0) + (shared ? p.out_row0_shared : 0));
+              bulk_commit_group();
+            }
+          } else {
+            __syncwarp();
+            if (probe) MOE_TRACE(MODE, i, 9);
+            uint4 rowv[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) rowv[c] = *reinterpret_cast<const uint4*>(tile + lane * 32 + 8 * c);
+            if (probe) MOE_TRACE(MODE, i, 10);
+            if (tok < un.ntok) store_row32(out_base + row * ld + c0, cols - c0, rowv);
+          }
+          if (probe) MOE_TRACE(MODE, i, 11);
         }
       }
       tc_fence_before();
@@ -554,6 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
     }
   }
 
+  if (warp >= 2 && lane == 0) bulk_wait_group_all();  // epilogue stores complete
   __syncthreads();
   if (warp == 0 && lane == 0 && first) {
     // wait for any stage fill that was issued but never observed complete
@@ -590,6 +626,22 @@ EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(ptr);
   }
   return fn;
+}
+
+// bf16 row-major [rows, cols] as the destination of 32 x 32 TMA stores (no
+// swizzle: the epilogue tile is dense).
+bool make_store_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  memset(m, 0, sizeof(*m));
+  if (!base || rows == 0 || cols == 0) return true;  // never referenced
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // bf16 row-major [rows, cols] viewed as a 2-D tensor map with a box of
@@ -659,8 +711,11 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
             make_tmap(&g1.a0_shared, a.Ws1, (uint64_t)p.nsF, p.d, 128) &&
             make_tmap(&g1.a1_shared, a.Ws3, (uint64_t)p.nsF, p.d, 128) &&
             make_tmap(&g1.b_routed, a.x_perm, (uint64_t)p.R, p.d, kTokBox) &&
-            make_tmap(&g1.b_shared, p.ns ? a.x : nullptr, (uint64_t)p.T, p.d, kTokBox);
+            make_tmap(&g1.b_shared, p.ns ? a.x : nullptr, (uint64_t)p.T, p.d, kTokBox) &&
+            make_store_tmap(&g1.o_routed, a.h_perm, (uint64_t)p.R, p.F) &&
+            make_store_tmap(&g1.o_shared, p.ns ? a.h_sh : nullptr, (uint64_t)p.T, p.nsF);
   if (!ok) return cudaErrorInvalidValue;
+  g1.out_row0_shared = 0;
   g1.unit_base = a.unit_base1;
   g1.grp_row0 = a.grp_row0;
   g1.grp_rows = a.grp_rows;
@@ -688,8 +743,11 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   ok = make_tmap(&g2.a0_routed, a.W2, (uint64_t)p.N * p.d, p.F, 128) &&
        make_tmap(&g2.a0_shared, a.Ws2, (uint64_t)p.d, p.nsF, 128) &&
        make_tmap(&g2.b_routed, a.h_perm, (uint64_t)p.R, p.F, kTokBox) &&
-       make_tmap(&g2.b_shared, p.ns ? a.h_sh : nullptr, (uint64_t)p.T, p.nsF, kTokBox);
+       make_tmap(&g2.b_shared, p.ns ? a.h_sh : nullptr, (uint64_t)p.T, p.nsF, kTokBox) &&
+       make_store_tmap(&g2.o_routed, a.y_rows, (uint64_t)(p.R + p.T), p.d) &&
+       make_store_tmap(&g2.o_shared, a.y_rows, (uint64_t)(p.R + p.T), p.d);
   if (!ok) return cudaErrorInvalidValue;
+  g2.out_row0_shared = (int)p.R;
   g2.unit_base = a.unit_base2;
   g2.grp_row0 = a.grp_row0;
   g2.grp_rows = a.grp_rows;
@@ -714,12 +772,12 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
 }  // namespace moe
 
 #ifdef MOE_UNIT_TRACE
-// Copies the unit trace ([2][kTraceCtas][kTraceUnits][8] u64) to host memory
+// Copies the unit trace ([2][kTraceCtas][kTraceUnits][16] u64) to host memory
 // and clears it (trace builds only).
 extern "C" MOE_API int moe_unit_trace_read(void* host_dst) {
   cudaError_t e = cudaMemcpyFromSymbol(host_dst, moe::g_unit_trace, sizeof(moe::g_unit_trace));
   if (e != cudaSuccess) return (int)e;
-  static unsigned long long zeros[2 * moe::kTraceCtas * moe::kTraceUnits * 8];
+  static unsigned long long zeros[2 * moe::kTraceCtas * moe::kTraceUnits * 16];
   return (int)cudaMemcpyToSymbol(moe::g_unit_trace, zeros, sizeof(zeros));
 }
 #endif
