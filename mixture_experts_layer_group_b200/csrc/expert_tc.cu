@@ -50,7 +50,6 @@
 // Every mbarrier wait is bounded; on a timeout a CTA records
 // MOE_DEV_WAIT_TIMEOUT, drains its own copies and MMAs (bounded again),
 // frees its tensor memory and exits.
-#include <cuda.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -611,54 +610,14 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// bf16 row-major [rows, cols] as the destination of 32 x 32 TMA stores (no
-// swizzle: the epilogue tile is dense).
-bool make_store_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
-  memset(m, 0, sizeof(*m));
-  if (!base || rows == 0 || cols == 0) return true;  // never referenced
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {32, 32};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// bf16 row-major [rows, cols] viewed as a 2-D tensor map with a box of
-// 64 columns x box_rows rows and 128-byte swizzle. Rows/columns beyond the
-// tensor read as zero.
+// Token / weight operand: 64 columns x box_rows rows, 128-byte swizzle.
 bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  memset(m, 0, sizeof(*m));
-  if (!base || rows == 0 || cols == 0) return true;  // never referenced
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_tmap_bf16(m, base, rows, cols, kBK, box_rows, true);
+}
+
+// Destination of the epilogue's dense 32 x 32 tile stores.
+bool make_store_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  return make_tmap_bf16(m, base, rows, cols, 32, 32, false);
 }
 
 template <int MODE>

@@ -139,7 +139,8 @@ moe_status check_ws(const Layout& L, void* ws, size_t ws_bytes, size_t need) {
 
 moe_status run_router(const Problem& p, const Layout& L, const void* x, const void* W_r,
                       const float* b, int32_t* idx, float* gates, void* ws, cudaStream_t s) {
-  cudaError_t e = launch_router(p, x, W_r, b, at<float>(ws, L.logits), router_scratch_bytes(p), idx, gates, s);
+  cudaError_t e = launch_router(p, x, W_r, b, at<float>(ws, L.logits), router_scratch_bytes(p), idx, gates,
+                                at<unsigned>(ws, L.status), s);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 

@@ -66,7 +66,7 @@ extern "C" moe_status moe_route_noalloc(const moe_cfg* cfg, int64_t T, const voi
   cudaError_t e = scratch_address(&scratch);
   if (e == cudaSuccess)
     e = launch_router(p, x, W_r, b, static_cast<float*>(scratch), kNoallocScratchBytes, topk_idx, gates,
-                      static_cast<cudaStream_t>(stream));
+                      nullptr, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     record_cuda_error(e);
     return MOE_ERR_CUDA;

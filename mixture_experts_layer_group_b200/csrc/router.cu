@@ -1,10 +1,11 @@
-// Router: z = x W_r^T on CUDA cores, then score, group-limited top-k and
-// gates by warp shuffles (router steps of the "All 19 steps" list on the
+// Router: z = x W_r^T (fp32 layers on CUDA cores here; bf16 layers on the
+// tensor cores, router_tc.cu), then score, group-limited top-k and gates by
+// warp shuffles (router steps of the "All 19 steps" list on the
 // "DeepSeek-V3.2-Exp · Mixture of experts" page; the softmax top-k variant is
 // the GShard router of the "DeepSeekMoE" walkthrough, Step 2).
 //
-// Logits are accumulated in fp32 over 32-element K chunks and carried across
-// chunks in fp64, which keeps the logit error near 1e-7 at d = 7168 (a plain
+// The CUDA-core logits are accumulated in fp32 over 32-element K chunks and
+// carried across chunks in fp64, which keeps the logit error near 1e-7 at d = 7168 (a plain
 // fp32 running sum is an order of magnitude worse and would turn near-ties
 // into routing differences). bf16 products are exact in fp32. When the
 // token count alone gives too few CTAs (decode), K is split into S ranges
@@ -322,10 +323,14 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
 }  // namespace
 
 int router_k_splits(const Problem& p) {
-  // enough CTAs to fill the SMs twice, each split keeping >= 4 K chunks
-  const int64_t base = (int64_t)((p.N + kLBN - 1) / kLBN) * ((p.T + kLBT - 1) / kLBT);
-  int64_t S = base > 0 ? (2 * (int64_t)kRouterTargetSms) / base : 1;
-  const int64_t by_k = p.d / (4 * kLBK);
+  // enough CTAs to fill the SMs (tensor cores: once, one CTA per SM; SIMT:
+  // twice), each split keeping >= 4 K chunks
+  const bool tc = p.dtype == MOE_BF16;
+  const int64_t tn = tc ? kRtcExperts : kLBN, tt = tc ? kRtcTokens : kLBT, kc = tc ? kRtcChunk : kLBK;
+  const int64_t base = (int64_t)((p.N + tn - 1) / tn) * ((p.T + tt - 1) / tt);
+  const int64_t target = (tc ? 1 : 2) * (int64_t)kRouterTargetSms;
+  int64_t S = base > 0 ? target / base : 1;
+  const int64_t by_k = p.d / (4 * kc);
   if (S > by_k) S = by_k;
   if (S > 16) S = 16;
   return S < 1 ? 1 : (int)S;
@@ -337,21 +342,23 @@ size_t router_scratch_bytes(const Problem& p) {
 
 cudaError_t launch_router(const Problem& p, const void* x, const void* W_r, const float* b,
                           float* logits, size_t logits_bytes, int32_t* idx, float* gates,
-                          cudaStream_t s) {
+                          unsigned* status, cudaStream_t s) {
   // as many K splits as router_k_splits(p) asks for and the scratch can hold
   const size_t plane = (size_t)p.T * (size_t)p.N * sizeof(float);
   int S = router_k_splits(p);
   if ((size_t)S * plane > logits_bytes) S = (int)(logits_bytes / plane);
   if (S < 1) return cudaErrorInvalidValue;
-  const int k_len = ((p.d + S - 1) / S + kLBK - 1) / kLBK * kLBK;
-  dim3 grid((unsigned)((p.N + kLBN - 1) / kLBN), (unsigned)((p.T + kLBT - 1) / kLBT), (unsigned)S);
-  if (p.dtype == MOE_BF16)
-    router_logits_kernel<__nv_bfloat16><<<grid, kLThreads, 0, s>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)W_r, p.T, p.N, p.d, k_len, logits);
-  else
+  cudaError_t err;
+  if (p.dtype == MOE_BF16) {
+    const int k_len = ((p.d + S - 1) / S + kRtcChunk - 1) / kRtcChunk * kRtcChunk;
+    err = launch_router_logits_tc(p, x, W_r, S, k_len, logits, status, s);
+  } else {
+    const int k_len = ((p.d + S - 1) / S + kLBK - 1) / kLBK * kLBK;
+    dim3 grid((unsigned)((p.N + kLBN - 1) / kLBN), (unsigned)((p.T + kLBT - 1) / kLBT), (unsigned)S);
     router_logits_kernel<float><<<grid, kLThreads, 0, s>>>((const float*)x, (const float*)W_r, p.T,
                                                            p.N, p.d, k_len, logits);
-  cudaError_t err = cudaGetLastError();
+    err = cudaGetLastError();
+  }
   if (err != cudaSuccess) return err;
 
   SelectArgs a{logits, S, b, p.T, p.N, p.k, p.G, p.TG, p.score_fn, p.group_score, p.normalize,
