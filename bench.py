@@ -363,6 +363,43 @@ def run_reference(args, rank, world):
             "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_router_only(args):
+    """moe_route alone (router logits + selection) on the config's x, W_r, b:
+    for profiling the router without the expert weights on the device."""
+    import torch
+    import mixture_experts_layer_group_b200 as moe
+    from mixture_experts_layer_group_b200 import build as lib_build
+    from moe_inputs import build as gen_build
+    from moe_inputs import device as mdev
+
+    lib_build.build()
+    gen_build.build()
+    s = mi.SHAPES[args.config]
+    x = mdev.device_tensor(s, "x")
+    W_r = mdev.device_tensor(s, "W_r")
+    b = mdev.device_tensor(s, "b") if s.bias else None
+    cfg = moe.make_cfg(s.d, s.d_ff, s.n_routed, s.n_shared, s.top_k, s.n_groups, s.topk_groups, s.score,
+                       s.normalize, s.route_scale, s.group_score, s.dtype)
+    ws = torch.empty(moe.workspace_size(cfg, s.T), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((s.T, s.top_k), dtype=torch.int32, device="cuda")
+    gates = torch.empty((s.T, s.top_k), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        moe.route(cfg, s.T, x, W_r, b, idx, gates, ws, stream=stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        moe.route(cfg, s.T, x, W_r, b, idx, gates, ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 2.0 * s.T * s.n_routed * s.d
+    return {"metric": "router tokens/s (moe_route alone)", "value": round(s.T / (ms * 1e-3), 1),
+            "unit": "tokens/s", "ms_per_step": round(ms, 4), "steps": args.steps, "warmup": args.warmup,
+            "router_tflops": round(flops / (ms * 1e-3) / 1e12, 2), "config": {"workload": s.name, "T": s.T}}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -372,10 +409,15 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage", default="layer", choices=["layer", "router"],
+                    help="router: time moe_route alone (profiling aid; 1 GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local_rank = rank_env()
+    if args.stage == "router":
+        print(json.dumps(run_router_only(args)), flush=True)
+        return 0
     if args.impl == "reference":
         out = run_reference(args, rank, world)
         if out:

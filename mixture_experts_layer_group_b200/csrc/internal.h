@@ -71,23 +71,16 @@ struct DispatchBuffers {
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                     uint32_t box_rows, bool swizzle128);
 
-// Router: logits (tensor cores for bf16, SIMT for fp32) then selection.
-// With router_scratch_bytes(p) bytes of logits scratch the router uses
-// router_k_splits(p) K ranges; with less (at least T * N * 4) it uses as
-// many as fit. `status` (may be null) collects MOE_DEV_* bits.
+// Router: logits (FP32 pipes) then selection. With router_scratch_bytes(p)
+// bytes of logits scratch the router uses router_k_splits(p) K ranges; with
+// less (at least T * N * 4) it uses as many as fit. `status` (may be null)
+// is reserved for MOE_DEV_* bits.
 constexpr int kRouterTargetSms = 148;
 int router_k_splits(const Problem& p);
 size_t router_scratch_bytes(const Problem& p);
 cudaError_t launch_router(const Problem& p, const void* x, const void* W_r, const float* b,
                           float* logits, size_t logits_bytes, int32_t* idx, float* gates,
                           unsigned* status, cudaStream_t s);
-// The tensor-core logits kernel alone: S K-range planes of fp32 partial
-// logits [S, T, N], k_len a multiple of 64.
-constexpr int kRtcTokens = 128;   // tokens per CTA (UMMA M)
-constexpr int kRtcExperts = 64;   // experts per CTA (UMMA N)
-constexpr int kRtcChunk = 64;     // K per stage and per fp64 carry
-cudaError_t launch_router_logits_tc(const Problem& p, const void* x, const void* W_r, int S, int k_len,
-                                    float* logits, unsigned* status, cudaStream_t s);
 
 // Histogram / scan / scatter; bm, bn1, bn2 select the GEMM tile grid that
 // the unit tables describe.

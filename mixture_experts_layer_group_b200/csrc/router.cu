@@ -1,11 +1,10 @@
-// Router: z = x W_r^T (fp32 layers on CUDA cores here; bf16 layers on the
-// tensor cores, router_tc.cu), then score, group-limited top-k and gates by
-// warp shuffles (router steps of the "All 19 steps" list on the
+// Router: z = x W_r^T on the FP32 pipes (CUDA cores), then score,
+// group-limited top-k and gates by warp shuffles (router steps of the "All 19 steps" list on the
 // "DeepSeek-V3.2-Exp · Mixture of experts" page; the softmax top-k variant is
 // the GShard router of the "DeepSeekMoE" walkthrough, Step 2).
 //
-// The CUDA-core logits are accumulated in fp32 over 32-element K chunks and
-// carried across chunks in fp64, which keeps the logit error near 1e-7 at d = 7168 (a plain
+// Logits are accumulated in fp32 over 128-element K runs and carried across
+// runs in fp64, which keeps the logit error near 1e-7 at d = 7168 (a plain
 // fp32 running sum is an order of magnitude worse and would turn near-ties
 // into routing differences). bf16 products are exact in fp32. When the
 // token count alone gives too few CTAs (decode), K is split into S ranges
@@ -22,56 +21,75 @@ namespace {
 
 constexpr int kLBT = 64;   // tokens per CTA tile
 constexpr int kLBN = 64;   // experts per CTA tile
-constexpr int kLBK = 32;   // K chunk
+constexpr int kLBK = 32;   // K chunk (one shared-memory buffer)
+constexpr int kLCarry = 4; // chunks summed in fp32 before each fp64 carry (128 K elements)
 constexpr int kLPitch = kLBK + 4;  // smem row pitch (floats): conflict-free strided float4 reads
-constexpr int kLThreads = 256;
+constexpr int kLThreads = 128;
+constexpr int kLTA = kLBT / 8;   // tokens per thread (8 thread rows)
+constexpr int kLTB = kLBN / 16;  // experts per thread (16 thread columns)
+constexpr int kLBufFloats = (kLBT + kLBN) * kLPitch;
+constexpr int kLSmemBytes = 2 * kLBufFloats * (int)sizeof(float);
+constexpr int kLCtasPerSm = 2;
 
 template <typename TIn>
 struct Vec16 {
   static constexpr int kElems = 16 / sizeof(TIn);
 };
 
-// Loads 16 bytes of row `row` (row pitch d) at column k (zero outside
-// [0, rows) x [0, k_end)).
+// 16 bytes of row `row` (row pitch d) at column k, zero outside
+// [0, rows) x [0, k_end).
 template <typename TIn>
-MOE_DEV void load_vec(const TIn* base, int64_t rows, int k_end, int d, int64_t row, int k, float* out) {
-  constexpr int E = Vec16<TIn>::kElems;
-  if (row < rows && k < k_end) {
-    uint4 v = *reinterpret_cast<const uint4*>(base + row * (int64_t)d + k);
-    if constexpr (sizeof(TIn) == 2) {
-      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&v);
+MOE_DEV uint4 load_raw(const TIn* base, int64_t rows, int k_end, int d, int64_t row, int k) {
+  if (row < rows && k < k_end) return __ldg(reinterpret_cast<const uint4*>(base + row * (int64_t)d + k));
+  return make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Widens 16 raw bytes to fp32 (exact for bf16) and stores them at dst.
+template <typename TIn>
+MOE_DEV void store_widened(float* dst, uint4 v) {
+  if constexpr (sizeof(TIn) == 2) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int i = 0; i < E; ++i) out[i] = __bfloat162float(h[i]);
-    } else {
-      const float* f = reinterpret_cast<const float*>(&v);
-#pragma unroll
-      for (int i = 0; i < E; ++i) out[i] = f[i];
+    for (int i = 0; i < 4; i += 2) {
+      *reinterpret_cast<float4*>(dst + 2 * i) =
+          make_float4(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u),
+                      __uint_as_float(w[i + 1] << 16), __uint_as_float(w[i + 1] & 0xffff0000u));
     }
   } else {
-#pragma unroll
-    for (int i = 0; i < E; ++i) out[i] = 0.f;
+    *reinterpret_cast<uint4*>(dst) = v;
   }
 }
 
-// One CTA computes a 64-token x 64-expert tile of logits. Thread (tx, ty)
-// owns tokens ty + 16a and experts tx + 16b (a, b in 0..3) so that the
-// strided float4 reads of each K step are bank-conflict free.
+// One CTA computes a 64-token x 64-expert tile of logits over one K range
+// on the FP32 pipes. Thread (tx, ty) owns tokens ty + 8a (a < 8) and
+// experts tx + 16b (b < 4): per 4 K elements it reads 8 + 4 float4 from
+// shared memory (one wavefront each: broadcast within the warp and
+// conflict-free with the padded pitch) for 128 FMAs. Operand tiles are widened to fp32 once, when staged;
+// the two shared-memory buffers alternate so each chunk needs one barrier,
+// and the global loads of chunk c + 2 are in flight while chunk c computes.
+// Two CTAs share an SM. The products go through the paired FP32 FMA
+// (__ffma2_rn: one instruction, two lanes of fp32 FMA), which halves the
+// issue slots the arithmetic needs: acc holds the running sums over the even
+// and the odd K positions of each (token, expert), added at each carry.
 template <typename TIn>
-__global__ void __launch_bounds__(kLThreads) router_logits_kernel(const TIn* __restrict__ x,
-                                                                  const TIn* __restrict__ W,
-                                                                  int64_t T, int N, int d, int k_len,
-                                                                  float* __restrict__ logits) {
+__global__ void __launch_bounds__(kLThreads, kLCtasPerSm) router_logits_kernel(const TIn* __restrict__ x,
+                                                                     const TIn* __restrict__ W,
+                                                                     int64_t T, int N, int d, int k_len,
+                                                                     float* __restrict__ logits) {
   constexpr int E = Vec16<TIn>::kElems;          // elements per 16-byte vector
   constexpr int kVecPerRow = kLBK / E;           // vectors per row per chunk
-  constexpr int kVecPerTile = kLBT * kVecPerRow; // vectors per operand tile
-  constexpr int kLoads = kVecPerTile / kLThreads;
-  static_assert(kVecPerTile % kLThreads == 0, "tile / thread mismatch");
+  constexpr int kXLoads = kLBT * kVecPerRow / kLThreads;
+  constexpr int kWLoads = (kLBN * kVecPerRow + kLThreads - 1) / kLThreads;
+  static_assert(kLBT * kVecPerRow % kLThreads == 0, "tile / threads");
+  constexpr int kWVecs = kLBN * kVecPerRow;      // W vectors per chunk (may be < threads)
 
-  __shared__ __align__(16) float xs[kLBT][kLPitch];
-  __shared__ __align__(16) float ws[kLBN][kLPitch];
+  extern __shared__ __align__(16) float lsm[];
 
   const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
+  // a warp covers 4 token rows x 8 expert rows of the 8 x 16 thread grid, so
+  // each float4 read touches 4 (x) or 8 (W) distinct rows: one wavefront
+  const int warp = tid >> 5, lane = tid & 31;
+  const int tx = (warp & 1) * 8 + (lane & 7), ty = (warp >> 1) * 4 + (lane >> 3);
   const int64_t t0 = (int64_t)blockIdx.y * kLBT;
   const int64_t e0 = (int64_t)blockIdx.x * kLBN;
   // this CTA's K range [k_begin, k_end) and its partial-logit plane
@@ -79,78 +97,91 @@ __global__ void __launch_bounds__(kLThreads) router_logits_kernel(const TIn* __r
   const int k_end = min(d, k_begin + k_len);
   logits += (int64_t)blockIdx.z * T * N;
 
-  float xr[kLoads][E], wr[kLoads][E];
+  uint4 xr[kXLoads], wr[kWLoads];
   auto fetch = [&](int kbase) {
 #pragma unroll
-    for (int i = 0; i < kLoads; ++i) {
-      int v = tid + i * kLThreads;
-      int row = v / kVecPerRow, kv = (v % kVecPerRow) * E;
-      load_vec<TIn>(x, T, k_end, d, t0 + row, kbase + kv, xr[i]);
-      load_vec<TIn>(W, N, k_end, d, e0 + row, kbase + kv, wr[i]);
+    for (int i = 0; i < kXLoads; ++i) {
+      const int v = tid + i * kLThreads;
+      xr[i] = load_raw<TIn>(x, T, k_end, d, t0 + v / kVecPerRow, kbase + (v % kVecPerRow) * E);
+    }
+#pragma unroll
+    for (int i = 0; i < kWLoads; ++i) {
+      const int v = tid + i * kLThreads;
+      if (v < kWVecs) wr[i] = load_raw<TIn>(W, N, k_end, d, e0 + v / kVecPerRow, kbase + (v % kVecPerRow) * E);
     }
   };
-  auto stash = [&]() {
+  auto stash = [&](int buf) {
+    float* xs = lsm + buf * kLBufFloats;
+    float* ws = xs + kLBT * kLPitch;
 #pragma unroll
-    for (int i = 0; i < kLoads; ++i) {
-      int v = tid + i * kLThreads;
-      int row = v / kVecPerRow, kv = (v % kVecPerRow) * E;
+    for (int i = 0; i < kXLoads; ++i) {
+      const int v = tid + i * kLThreads;
+      store_widened<TIn>(xs + (v / kVecPerRow) * kLPitch + (v % kVecPerRow) * E, xr[i]);
+    }
 #pragma unroll
-      for (int j = 0; j < E; j += 4) {
-        *reinterpret_cast<float4*>(&xs[row][kv + j]) =
-            make_float4(xr[i][j], xr[i][j + 1], xr[i][j + 2], xr[i][j + 3]);
-        *reinterpret_cast<float4*>(&ws[row][kv + j]) =
-            make_float4(wr[i][j], wr[i][j + 1], wr[i][j + 2], wr[i][j + 3]);
-      }
+    for (int i = 0; i < kWLoads; ++i) {
+      const int v = tid + i * kLThreads;
+      if (v < kWVecs) store_widened<TIn>(ws + (v / kVecPerRow) * kLPitch + (v % kVecPerRow) * E, wr[i]);
     }
   };
 
-  double total[4][4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) total[a][b] = 0.0;
 
-  const int nk = (k_end - k_begin + kLBK - 1) / kLBK;
-  fetch(k_begin);
+  double total[kLTA][kLTB];
+  float2 acc[kLTA][kLTB];
+#pragma unroll
+  for (int a = 0; a < kLTA; ++a)
+#pragma unroll
+    for (int b = 0; b < kLTB; ++b) {
+      total[a][b] = 0.0;
+      acc[a][b] = make_float2(0.f, 0.f);
+    }
+
+  const int nk = k_end > k_begin ? (k_end - k_begin + kLBK - 1) / kLBK : 0;
+  if (nk > 0) {
+    fetch(k_begin);
+    stash(0);
+    __syncthreads();
+    if (nk > 1) fetch(k_begin + kLBK);
+  }
   for (int kc = 0; kc < nk; ++kc) {
-    __syncthreads();
-    stash();
-    __syncthreads();
-    if (kc + 1 < nk) fetch(k_begin + (kc + 1) * kLBK);
-    float acc[4][4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+    const float* xs = lsm + (kc & 1) * kLBufFloats;
+    const float* ws = xs + kLBT * kLPitch;
 #pragma unroll
     for (int kk = 0; kk < kLBK; kk += 4) {
-      float4 xv[4], wv[4];
+      float4 wv[kLTB];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) xv[a] = *reinterpret_cast<const float4*>(&xs[ty + 16 * a][kk]);
+      for (int b = 0; b < kLTB; ++b) wv[b] = *reinterpret_cast<const float4*>(ws + (tx + 16 * b) * kLPitch + kk);
 #pragma unroll
-      for (int b = 0; b < 4; ++b) wv[b] = *reinterpret_cast<const float4*>(&ws[tx + 16 * b][kk]);
+      for (int a = 0; a < kLTA; ++a) {
+        const float4 xv = *reinterpret_cast<const float4*>(xs + (ty + 8 * a) * kLPitch + kk);
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+        for (int b = 0; b < kLTB; ++b) {
+          acc[a][b] = __ffma2_rn(make_float2(xv.x, xv.y), make_float2(wv[b].x, wv[b].y), acc[a][b]);
+          acc[a][b] = __ffma2_rn(make_float2(xv.z, xv.w), make_float2(wv[b].z, wv[b].w), acc[a][b]);
+        }
+      }
+    }
+    if ((kc + 1) % kLCarry == 0 || kc + 1 == nk) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          acc[a][b] = fmaf(xv[a].x, wv[b].x, acc[a][b]);
-          acc[a][b] = fmaf(xv[a].y, wv[b].y, acc[a][b]);
-          acc[a][b] = fmaf(xv[a].z, wv[b].z, acc[a][b]);
-          acc[a][b] = fmaf(xv[a].w, wv[b].w, acc[a][b]);
+      for (int a = 0; a < kLTA; ++a)
+#pragma unroll
+        for (int b = 0; b < kLTB; ++b) {
+          total[a][b] += (double)acc[a][b].x + (double)acc[a][b].y;
+          acc[a][b] = make_float2(0.f, 0.f);
         }
     }
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) total[a][b] += (double)acc[a][b];
+    // the other buffer was last read before the previous barrier
+    if (kc + 1 < nk) stash((kc + 1) & 1);
+    __syncthreads();
+    if (kc + 2 < nk) fetch(k_begin + (kc + 2) * kLBK);
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    int64_t t = t0 + ty + 16 * a;
+  for (int a = 0; a < kLTA; ++a) {
+    const int64_t t = t0 + ty + 8 * a;
     if (t >= T) continue;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      int64_t e = e0 + tx + 16 * b;
+    for (int b = 0; b < kLTB; ++b) {
+      const int64_t e = e0 + tx + 16 * b;
       if (e < N) logits[t * N + e] = (float)total[a][b];
     }
   }
@@ -323,17 +354,24 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
 }  // namespace
 
 int router_k_splits(const Problem& p) {
-  // enough CTAs to fill the SMs (tensor cores: once, one CTA per SM; SIMT:
-  // twice), each split keeping >= 4 K chunks
-  const bool tc = p.dtype == MOE_BF16;
-  const int64_t tn = tc ? kRtcExperts : kLBN, tt = tc ? kRtcTokens : kLBT, kc = tc ? kRtcChunk : kLBK;
-  const int64_t base = (int64_t)((p.N + tn - 1) / tn) * ((p.T + tt - 1) / tt);
-  const int64_t target = (tc ? 1 : 2) * (int64_t)kRouterTargetSms;
-  int64_t S = base > 0 ? target / base : 1;
-  const int64_t by_k = p.d / (4 * kc);
-  if (S > by_k) S = by_k;
-  if (S > 16) S = 16;
-  return S < 1 ? 1 : (int)S;
+  // The split count with the fewest CTA waves per unit of K work (a split adds a T x N plane for the selection kernel to read, so
+  // a larger count must win by more than 1%), each split keeping >= 4 chunks.
+  const int64_t base = (int64_t)((p.N + kLBN - 1) / kLBN) * ((p.T + kLBT - 1) / kLBT);
+  if (base <= 0) return 1;
+  int64_t max_s = p.d / (4 * kLBK);
+  if (max_s > 16) max_s = 16;
+  int best = 1;
+  double best_cost = 1e30;
+  for (int64_t S = 1; S <= max_s; ++S) {
+    const int64_t slots = (int64_t)kRouterTargetSms * kLCtasPerSm;
+    const int64_t waves = (base * S + slots - 1) / slots;
+    const double cost = (double)waves / (double)S;
+    if (cost < best_cost * 0.99) {
+      best_cost = cost;
+      best = (int)S;
+    }
+  }
+  return best;
 }
 
 size_t router_scratch_bytes(const Problem& p) {
@@ -343,22 +381,34 @@ size_t router_scratch_bytes(const Problem& p) {
 cudaError_t launch_router(const Problem& p, const void* x, const void* W_r, const float* b,
                           float* logits, size_t logits_bytes, int32_t* idx, float* gates,
                           unsigned* status, cudaStream_t s) {
+  (void)status;
   // as many K splits as router_k_splits(p) asks for and the scratch can hold
   const size_t plane = (size_t)p.T * (size_t)p.N * sizeof(float);
   int S = router_k_splits(p);
   if ((size_t)S * plane > logits_bytes) S = (int)(logits_bytes / plane);
   if (S < 1) return cudaErrorInvalidValue;
-  cudaError_t err;
-  if (p.dtype == MOE_BF16) {
-    const int k_len = ((p.d + S - 1) / S + kRtcChunk - 1) / kRtcChunk * kRtcChunk;
-    err = launch_router_logits_tc(p, x, W_r, S, k_len, logits, status, s);
-  } else {
-    const int k_len = ((p.d + S - 1) / S + kLBK - 1) / kLBK * kLBK;
-    dim3 grid((unsigned)((p.N + kLBN - 1) / kLBN), (unsigned)((p.T + kLBT - 1) / kLBT), (unsigned)S);
-    router_logits_kernel<float><<<grid, kLThreads, 0, s>>>((const float*)x, (const float*)W_r, p.T,
-                                                           p.N, p.d, k_len, logits);
-    err = cudaGetLastError();
+  const int k_len = ((p.d + S - 1) / S + kLBK - 1) / kLBK * kLBK;
+  dim3 grid((unsigned)((p.N + kLBN - 1) / kLBN), (unsigned)((p.T + kLBT - 1) / kLBT), (unsigned)S);
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (configured_device != dev) {
+    err = cudaFuncSetAttribute(router_logits_kernel<__nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kLSmemBytes);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(router_logits_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kLSmemBytes);
+    if (err != cudaSuccess) return err;
+    configured_device = dev;
   }
+  if (p.dtype == MOE_BF16)
+    router_logits_kernel<__nv_bfloat16><<<grid, kLThreads, kLSmemBytes, s>>>(
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)W_r, p.T, p.N, p.d, k_len, logits);
+  else
+    router_logits_kernel<float><<<grid, kLThreads, kLSmemBytes, s>>>((const float*)x, (const float*)W_r, p.T,
+                                                                     p.N, p.d, k_len, logits);
+  err = cudaGetLastError();
   if (err != cudaSuccess) return err;
 
   SelectArgs a{logits, S, b, p.T, p.N, p.k, p.G, p.TG, p.score_fn, p.group_score, p.normalize,
