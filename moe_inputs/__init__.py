@@ -92,6 +92,10 @@ SHAPES = {
 SHAPES["v3_profile_32e"] = LayerShape("v3_profile_32e", T=1024, d=7168, n_routed=32, n_shared=1, d_ff=2048,
                                       top_k=8, score="sigmoid", n_groups=8, topk_groups=4, normalize=True,
                                       route_scale=2.5, seed=5, bias=True)
+# Supplementary V3 prefill at T = 16384 (512 tokens per routed expert on
+# average): the same layer and seed with four times the tokens, which moves
+# the expert GEMMs from the HBM roofline to the tensor-core roofline.
+SHAPES["v3_prefill_t16k_bf16"] = SHAPES["v3_prefill_bf16"].with_(name="v3_prefill_t16k_bf16", T=16384)
 ORDER = ["gshard_tiny_f32", "dsmoe_2b_bf16", "v2_layer_bf16", "v3_prefill_bf16", "v3_decode_bf16"]
 
 

@@ -181,10 +181,10 @@ def test_abi_errors_on_device_buffers():
 # ------------------------------------------------------------- full size ----
 
 SAMPLES = {"gshard_tiny_f32": None, "dsmoe_2b_bf16": 64, "v2_layer_bf16": 16, "v3_prefill_bf16": 16,
-           "v3_decode_bf16": None}
+           "v3_decode_bf16": None, "v3_prefill_t16k_bf16": 16}
 
 
-@pytest.mark.parametrize("name", mi.ORDER)
+@pytest.mark.parametrize("name", mi.ORDER + ["v3_prefill_t16k_bf16"])
 def test_full_size_config(name):
     s = mi.SHAPES[name]
     w = mdev.device_all(s)
