@@ -32,8 +32,8 @@
 // CTAs of a pair except the MMA issuer, which only the first CTA has):
 //   warp 0      TMA producer (one lane). In CTA 0 it also takes unit ids and
 //               hands them to both CTAs through shared-memory rings. Stages
-//               are variable-size pieces (32 KB of weights + 4 KB per 32 token
-//               rows) of a 204 KB byte ring; the bytes of both CTAs complete
+//               are variable-size pieces (32 KB of weights + one token box of
+//               32, 64 or 128 rows, 4 / 8 / 16 KB) of a 208 KB byte ring; the bytes of both CTAs complete
 //               on CTA 0's stage barrier; weights read by one unit only are
 //               evict-first
 //   warp 1      TMEM owner (both CTAs, pair allocation) + UMMA issuer (CTA 0,
@@ -60,8 +60,9 @@ namespace {
 constexpr int kSlots = 8;                         // stages in flight at most
 constexpr int kBK = 64;                           // bf16 per K chunk: one 128 B swizzle row
 constexpr int kMaxTok = kTcBM;                    // tokens per unit (<= 256)
-constexpr int kTokBox = 32;                       // token rows per TMA box
+constexpr int kTokBox = 32;                       // token-row granule of a stage
 constexpr int kBoxBytes = kTokBox * kBK * 2;      // 4 KB
+constexpr int kTokMaps = 3;                       // token boxes of 32, 64 and 128 rows
 constexpr int kHalfBytes = 128 * kBK * 2;         // 16 KB: 128 weight rows of one half
 constexpr int kATileBytes = 2 * kHalfBytes;       // 32 KB: this CTA's rows of both halves
 constexpr int kMaxStageBytes = kATileBytes + (kMaxTok / 2 / kTokBox) * kBoxBytes;  // 48 KB
@@ -105,8 +106,8 @@ struct TcParams {
   CUtensorMap a1_routed;  // W3 [N*F, d]      | unused
   CUtensorMap a0_shared;  // Ws1 [nsF, d]     | Ws2 [d, nsF]
   CUtensorMap a1_shared;  // Ws3 [nsF, d]     | unused
-  CUtensorMap b_routed;   // x_perm [R, d]    | h_perm [R, F]
-  CUtensorMap b_shared;   // x [T, d]         | h_sh [T, nsF]
+  CUtensorMap b_routed[kTokMaps];  // x_perm [R, d] | h_perm [R, F]   (boxes of 32 / 64 / 128 rows)
+  CUtensorMap b_shared[kTokMaps];  // x [T, d]      | h_sh [T, nsF]
   CUtensorMap o_routed;   // h_perm [R, F]    | y_rows [R + T, d]   (32 x 32 store box)
   CUtensorMap o_shared;   // h_sh [T, nsF]    | y_rows [R + T, d]
   const int32_t* unit_base;  // [N + 2]: units before group g; [N + 1] = total
@@ -250,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.a0_routed);
-    tma_prefetch_desc(&p.b_routed);
+    for (int m = 0; m < kTokMaps; ++m) tma_prefetch_desc(&p.b_routed[m]);
     if (MODE == kSwiGLU) tma_prefetch_desc(&p.a1_routed);
   }
   if (warp == 1) {
@@ -338,13 +339,17 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         const int K = shared ? p.k_shared : p.k_routed;
         const int nk = (K + kBK - 1) / kBK;
         const int half_n = ((un.ntok + 15) & ~15) / 2;  // token rows per CTA
-        const int nbox = (half_n + kTokBox - 1) / kTokBox;
+        // one token box per stage, the smallest of 32 / 64 / 128 rows that
+        // covers this CTA's rows (the TMA engine's cost is per box, so a
+        // single box beats several small ones even with rows to spare)
+        const int tmap = half_n <= kTokBox ? 0 : (half_n <= 2 * kTokBox ? 1 : 2);
+        const int nbox = 1 << tmap;  // in 32-row granules
         const uint32_t tx = kATileBytes + nbox * kBoxBytes;
         const int rowA = (shared ? 0 : un.g * p.a_rows_per_expert) + un.f * p.tile_cols + rank_rows;
         const int rowB = __ldg(p.grp_row0 + un.g) + un.tok0 + (int)rank * half_n;
         const CUtensorMap* ta0 = shared ? &p.a0_shared : &p.a0_routed;
         const CUtensorMap* ta1 = MODE == kSwiGLU ? (shared ? &p.a1_shared : &p.a1_routed) : ta0;
-        const CUtensorMap* tb = shared ? &p.b_shared : &p.b_routed;
+        const CUtensorMap* tb = shared ? &p.b_shared[tmap] : &p.b_routed[tmap];
         const uint64_t pol = un.nchunks == 1 ? pol_once : pol_shared;
         MOE_TRACE(MODE, i, 0);
         MOE_TRACE_VAL(MODE, i, 7, (unsigned long long)un.ntok | ((unsigned long long)un.tok0 << 16) |
@@ -365,8 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           if (first) mbar_arrive_expect_tx(&sh.full[s], 2 * tx);  // this CTA's bytes and the peer's
           tma_load_2d_pair(a_dst, ta0, full_bar, kc * kBK, rowA, pol);
           tma_load_2d_pair(a_dst + kHalfBytes, ta1, full_bar, kc * kBK, rowA + half_rows, pol);
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d_pair(b_dst + b * kBoxBytes, tb, full_bar, kc * kBK, rowB + b * kTokBox, pol_shared);
+          tma_load_2d_pair(b_dst, tb, full_bar, kc * kBK, rowB, pol_shared);
         }
         MOE_TRACE(MODE, i, 1);
         if (!ok) break;
@@ -615,6 +619,13 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
   return make_tmap_bf16(m, base, rows, cols, kBK, box_rows, true);
 }
 
+// Token operand maps with boxes of 32, 64 and 128 rows.
+bool make_token_tmaps(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  for (int i = 0; i < kTokMaps; ++i)
+    if (!make_tmap(&m[i], base, rows, cols, (uint32_t)(kTokBox << i))) return false;
+  return true;
+}
+
 // Destination of the epilogue's dense 32 x 32 tile stores.
 bool make_store_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
   return make_tmap_bf16(m, base, rows, cols, 32, 32, false);
@@ -669,8 +680,8 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
             make_tmap(&g1.a1_routed, a.W3, (uint64_t)p.N * p.F, p.d, 128) &&
             make_tmap(&g1.a0_shared, a.Ws1, (uint64_t)p.nsF, p.d, 128) &&
             make_tmap(&g1.a1_shared, a.Ws3, (uint64_t)p.nsF, p.d, 128) &&
-            make_tmap(&g1.b_routed, a.x_perm, (uint64_t)p.R, p.d, kTokBox) &&
-            make_tmap(&g1.b_shared, p.ns ? a.x : nullptr, (uint64_t)p.T, p.d, kTokBox) &&
+            make_token_tmaps(g1.b_routed, a.x_perm, (uint64_t)p.R, p.d) &&
+            make_token_tmaps(g1.b_shared, p.ns ? a.x : nullptr, (uint64_t)p.T, p.d) &&
             make_store_tmap(&g1.o_routed, a.h_perm, (uint64_t)p.R, p.F) &&
             make_store_tmap(&g1.o_shared, p.ns ? a.h_sh : nullptr, (uint64_t)p.T, p.nsF);
   if (!ok) return cudaErrorInvalidValue;
@@ -701,8 +712,8 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   TcParams g2{};
   ok = make_tmap(&g2.a0_routed, a.W2, (uint64_t)p.N * p.d, p.F, 128) &&
        make_tmap(&g2.a0_shared, a.Ws2, (uint64_t)p.d, p.nsF, 128) &&
-       make_tmap(&g2.b_routed, a.h_perm, (uint64_t)p.R, p.F, kTokBox) &&
-       make_tmap(&g2.b_shared, p.ns ? a.h_sh : nullptr, (uint64_t)p.T, p.nsF, kTokBox) &&
+       make_token_tmaps(g2.b_routed, a.h_perm, (uint64_t)p.R, p.F) &&
+       make_token_tmaps(g2.b_shared, p.ns ? a.h_sh : nullptr, (uint64_t)p.T, p.nsF) &&
        make_store_tmap(&g2.o_routed, a.y_rows, (uint64_t)(p.R + p.T), p.d) &&
        make_store_tmap(&g2.o_shared, a.y_rows, (uint64_t)(p.R + p.T), p.d);
   if (!ok) return cudaErrorInvalidValue;
