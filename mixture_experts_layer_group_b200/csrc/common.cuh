@@ -335,6 +335,30 @@ MOE_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// 16 lanes x 256 bits, repeated over 4 column groups: thread i receives, for
+// column group r (columns 8r .. 8r + 7 from taddr), r[4r + 0..1] = lane
+// (base + i / 4), columns 8r + 2 (i % 4) + 0..1, and r[4r + 2..3] = lane
+// (base + 8 + i / 4), the same columns (the m16n8 accumulator layout).
+MOE_DEV void tmem_ld16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// Four 8 x 8 bf16 matrices, stored transposed: thread i holds element pair
+// (row i / 4, columns 2 (i % 4) + 0..1) of matrix m in register m; thread
+// 8 m + k gives the shared-memory address of stored row k of matrix m, which
+// receives column k (16 bytes).
+MOE_DEV void stmatrix_x4_trans(uint32_t smem_addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr),
+               "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
 MOE_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------ values --

@@ -526,36 +526,67 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         for (int j0 = 32 * sub; j0 < un.ntok; j0 += 32 * (kEpiWarps / 4)) {
           const int tok = j0 + lane;
           const int64_t row = row_base + tok;
-          // gate of this lane's token, spread to the column-owning lanes below
+          // gate of this lane's token, spread to the lanes that hold it below
           float my_gate = 1.0f;
           if (MODE == kGateDown && !shared && tok < un.ntok) my_gate = __ldg(p.gate_perm + row);
           if (leader && hh == 0 && j0 == 0) MOE_TRACE(MODE, i, 12);
-          float v[32];
-          {
-            uint32_t a[32];
-            tmem_ld32(t_q + hh * stride + j0, a);
+          // The block (32 features = this quadrant's TMEM lanes, x 32 tokens =
+          // columns j0..j0+31) in the m16n8 layout: lane half hf and column
+          // group r give this thread features 16 hf + 8 e + lane / 4 (e = 0, 1)
+          // and tokens 8 r + 2 (lane % 4) + 0..1, packed as bf16 pairs.
+          uint32_t pk[2][4][2];
+          const int tq = 2 * (lane & 3);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t a[16];
+            tmem_ld16x256b_x4(t_q + ((uint32_t)(16 * hf) << 16) + hh * stride + j0, a);
             if (MODE == kSwiGLU) {
-              uint32_t b[32];
-              tmem_ld32(t_q + stride + j0, b);  // u of the same feature
+              uint32_t b[16];
+              tmem_ld16x256b_x4(t_q + ((uint32_t)(16 * hf) << 16) + stride + j0, b);  // u of the same features
               tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const float g = __uint_as_float(a[j]);
-                v[j] = silu_tanh(g) * __uint_as_float(b[j]);
-              }
+              for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int x = 4 * r + 2 * e;
+                  pk[hf][r][e] = pack_bf16x2(silu_tanh(__uint_as_float(a[x])) * __uint_as_float(b[x]),
+                                             silu_tanh(__uint_as_float(a[x + 1])) * __uint_as_float(b[x + 1]));
+                }
             } else {
               tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]) * __shfl_sync(0xffffffffu, my_gate, j);
+              for (int r = 0; r < 4; ++r) {
+                const float g0 = __shfl_sync(0xffffffffu, my_gate, 8 * r + tq);
+                const float g1 = __shfl_sync(0xffffffffu, my_gate, 8 * r + tq + 1);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int x = 4 * r + 2 * e;
+                  pk[hf][r][e] = pack_bf16x2(__uint_as_float(a[x]) * g0, __uint_as_float(a[x + 1]) * g1);
+                }
+              }
             }
           }
           const bool probe = leader && hh == 0 && j0 == 0;
           if (probe) MOE_TRACE(MODE, i, 8);
-          // transpose through this warp's tile: lane = column -> row = token
+          // Transpose into this warp's [32 tokens][32 features] tile, 64-byte
+          // swizzled (16-byte chunk c of token row t sits at chunk c ^ ((t >> 1) & 3)),
+          // with four transposing matrix stores: matrix m of store (hf, rp) is
+          // column group r = 2 rp + m / 2 and feature octet e = m % 2.
           if (lane == 0) bulk_wait_group_read<0>();  // the previous block's store has read the tile
           __syncwarp();
+          const uint32_t tile_addr = smem_u32(tile);
+          {
+            const int m = lane >> 3, k = lane & 7;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) tile[j * 32 + lane] = __float2bfloat16_rn(v[j]);
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+              for (int rp = 0; rp < 2; ++rp) {
+                const int t = 8 * (2 * rp + (m >> 1)) + k;  // token row this lane addresses
+                const int c = 2 * hf + (m & 1);             // feature chunk
+                stmatrix_x4_trans(tile_addr + t * 64 + ((c ^ ((t >> 1) & 3)) << 4), pk[hf][2 * rp][0],
+                                  pk[hf][2 * rp][1], pk[hf][2 * rp + 1][0], pk[hf][2 * rp + 1][1]);
+              }
+          }
           const bool full_block = j0 + 32 <= un.ntok && c0 + 32 <= cols;
           if (full_block) {
             fence_proxy_async_smem();
@@ -572,7 +603,9 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
             if (probe) MOE_TRACE(MODE, i, 9);
             uint4 rowv[4];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) rowv[c] = *reinterpret_cast<const uint4*>(tile + lane * 32 + 8 * c);
+            for (int c = 0; c < 4; ++c)
+              rowv[c] = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(tile) + lane * 64 +
+                                                        ((c ^ ((lane >> 1) & 3)) << 4));
             if (probe) MOE_TRACE(MODE, i, 10);
             if (tok < un.ntok) store_row32(out_base + row * ld + c0, cols - c0, rowv);
           }
@@ -626,9 +659,9 @@ bool make_token_tmaps(CUtensorMap* m, const void* base, uint64_t rows, uint64_t 
   return true;
 }
 
-// Destination of the epilogue's dense 32 x 32 tile stores.
+// Destination of the epilogue's 32 x 32 tile stores (64-byte swizzled tile).
 bool make_store_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
-  return make_tmap_bf16(m, base, rows, cols, 32, 32, false);
+  return make_tmap_bf16_swz(m, base, rows, cols, 32, 32, 64);
 }
 
 template <int MODE>

@@ -70,6 +70,9 @@ struct DispatchBuffers {
 // base or an empty matrix gives a zeroed map that must not be used.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                     uint32_t box_rows, bool swizzle128);
+// The same with a swizzle of 0, 64 or 128 bytes.
+bool make_tmap_bf16_swz(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                        uint32_t box_rows, int swizzle_bytes);
 
 // Router: logits (FP32 pipes) then selection. With router_scratch_bytes(p)
 // bytes of logits scratch the router uses router_k_splits(p) K ranges; with

@@ -28,6 +28,11 @@ EncodeTiledFn encode_fn() {
 
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                     uint32_t box_rows, bool swizzle128) {
+  return make_tmap_bf16_swz(m, base, rows, cols, box_cols, box_rows, swizzle128 ? 128 : 0);
+}
+
+bool make_tmap_bf16_swz(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                        uint32_t box_rows, int swizzle_bytes) {
   memset(m, 0, sizeof(*m));
   if (!base || rows == 0 || cols == 0) return true;  // never referenced
   EncodeTiledFn enc = encode_fn();
@@ -38,8 +43,9 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE,
-             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-             swizzle128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : (swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE),
+             swizzle_bytes == 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
