@@ -394,6 +394,23 @@ def run_router_only(args):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
+    if args.stage == "bias":
+        # the balancing step on this batch's counts: route once, dispatch, then
+        # time moe_bias_update alone (N fp32 updates; launch-bound)
+        counts = torch.zeros(s.n_routed, dtype=torch.int32, device="cuda")
+        moe.dispatch(cfg, s.T, idx, counts, None, None, ws, stream=stream)
+        bias = b.clone() if b is not None else torch.zeros(s.n_routed, dtype=torch.float32, device="cuda")
+        for _ in range(args.warmup):
+            moe.bias_update(cfg, s.T, counts, 1e-3, bias, stream=stream)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            moe.bias_update(cfg, s.T, counts, 1e-3, bias, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / args.steps * 1e3
+        return {"metric": "moe_bias_update time", "value": round(us, 2), "unit": "us", "steps": args.steps,
+                "warmup": args.warmup, "higher_is_better": False, "config": {"workload": s.name, "N": s.n_routed}}
     flops = 2.0 * s.T * s.n_routed * s.d
     return {"metric": "router tokens/s (moe_route alone)", "value": round(s.T / (ms * 1e-3), 1),
             "unit": "tokens/s", "ms_per_step": round(ms, 4), "steps": args.steps, "warmup": args.warmup,
@@ -409,13 +426,13 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", default="layer", choices=["layer", "router"],
-                    help="router: time moe_route alone (profiling aid; 1 GPU)")
+    ap.add_argument("--stage", default="layer", choices=["layer", "router", "bias"],
+                    help="router: time moe_route alone; bias: time moe_bias_update (profiling aids; 1 GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local_rank = rank_env()
-    if args.stage == "router":
+    if args.stage in ("router", "bias"):
         print(json.dumps(run_router_only(args)), flush=True)
         return 0
     if args.impl == "reference":

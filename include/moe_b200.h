@@ -223,6 +223,28 @@ MOE_API moe_status moe_set_stage_events(void* const* events, int32_t n);
 MOE_API moe_status moe_route_noalloc(const moe_cfg* cfg, int64_t T, const void* x, const void* W_r,
                                      const float* b, int32_t* topk_idx, float* gates, void* stream);
 
+/*
+ * Auxiliary-loss-free load balancing: the per-batch bias nudge (grasp.study
+ * lesson on DeepSeek-V3's MoE design, section "3.2. Auxiliary-Loss-Free Load
+ * Balancing"; "The DeepSeekMoE Architecture.", configuration table row
+ * "balancing: aux-loss-free bias"). For every routed expert e:
+ *   b[e] -= gamma  if counts[e] > T * top_k / N   (overloaded)
+ *   b[e] += gamma  if counts[e] < T * top_k / N   (underloaded)
+ *   unchanged      otherwise
+ * (the comparison is exact, in integers; the update is one fp32 add).
+ *   counts [N] int32 in, device: the batch's (token, slot) pairs per expert,
+ *          as moe_dispatch writes them for the same T
+ *   gamma  the update rate (the pages give none; DeepSeek-V3 style values are
+ *          around 1e-3); must be finite
+ *   b      [N] fp32 in/out, device: the selection bias that moe_route and
+ *          moe_forward read
+ * Asynchronous on `stream`; no workspace; b is updated in place.
+ * Errors: MOE_ERR_INVALID_ARG for a bad cfg, null or misaligned pointers or a
+ * non-finite gamma; MOE_ERR_CUDA for a failed launch.
+ */
+MOE_API moe_status moe_bias_update(const moe_cfg* cfg, int64_t T, const int32_t* counts, float gamma, float* b,
+                                   void* stream);
+
 /* Human-readable name of a status code (static storage). */
 MOE_API const char* moe_status_string(moe_status status);
 

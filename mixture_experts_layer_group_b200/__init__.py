@@ -22,7 +22,7 @@ MOE_DEV_WAIT_TIMEOUT, MOE_DEV_BAD_EXPERT, MOE_DEV_DUP_EXPERT, MOE_DEV_TMEM_ALLOC
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE"}
 EXPORTS = ["moe_workspace_size", "moe_workspace_size_host", "moe_route", "moe_dispatch", "moe_forward",
-           "moe_forward_host", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc",
+           "moe_forward_host", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update",
            "moe_status_string", "moe_last_cuda_error"]
 STAGES = ["router", "dispatch", "gather", "gemm_swiglu", "gemm_gate", "combine"]
 
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
         L.moe_device_status.argtypes = [CFG, I64, P, SZ, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32), P]
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
         L.moe_route_noalloc.argtypes = [CFG, I64, P, P, P, P, P, P]
+        L.moe_bias_update.argtypes = [CFG, I64, P, ctypes.c_float, P, P]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_last_cuda_error.argtypes = []
@@ -134,6 +135,13 @@ def route_noalloc(cfg, T, x, W_r, b, topk_idx, gates, stream=None):
     bytes at most); calls that overlap on the GPU race on it."""
     _check("moe_route_noalloc", lib().moe_route_noalloc(ctypes.byref(cfg), T, _ptr(x), _ptr(W_r), _ptr(b),
                                                         _ptr(topk_idx), _ptr(gates), _stream(stream)))
+
+
+def bias_update(cfg, T, counts, gamma, b, stream=None):
+    """Auxiliary-loss-free balancing step: b[e] -= gamma where counts[e] exceeds
+    the mean load T * top_k / N, += gamma where it falls short (in place)."""
+    _check("moe_bias_update", lib().moe_bias_update(ctypes.byref(cfg), T, _ptr(counts), float(gamma), _ptr(b),
+                                                    _stream(stream)))
 
 
 def dispatch(cfg, T, topk_idx, counts, offsets, perm, ws, ws_bytes=None, stream=None):

@@ -96,6 +96,11 @@ SHAPES["v3_profile_32e"] = LayerShape("v3_profile_32e", T=1024, d=7168, n_routed
 # average): the same layer and seed with four times the tokens, which moves
 # the expert GEMMs from the HBM roofline to the tensor-core roofline.
 SHAPES["v3_prefill_t16k_bf16"] = SHAPES["v3_prefill_bf16"].with_(name="v3_prefill_t16k_bf16", T=16384)
+# V2-shaped layer with device-limited routing: the 160 routed experts spread
+# over 8 devices of 20, each token's experts drawn from the 3 devices holding
+# its highest affinities (group score = the device's best expert score).
+SHAPES["v2_device_limited_bf16"] = SHAPES["v2_layer_bf16"].with_(name="v2_device_limited_bf16", n_groups=8,
+                                                                   topk_groups=3, group_score="max")
 ORDER = ["gshard_tiny_f32", "dsmoe_2b_bf16", "v2_layer_bf16", "v3_prefill_bf16", "v3_decode_bf16"]
 
 

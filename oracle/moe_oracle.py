@@ -188,6 +188,25 @@ def permutation(idx: np.ndarray, n_routed: int):
     return counts, offsets, perm
 
 
+# ------------------------------------------------------------ balancing ----
+
+def bias_update(b: np.ndarray, counts: np.ndarray, T: int, k: int, gamma: float) -> np.ndarray:
+    """Auxiliary-loss-free load balancing, the per-batch bias nudge (grasp.study
+    lesson on DeepSeek-V3's MoE design, "3.2. Auxiliary-Loss-Free Load
+    Balancing": each expert's bias is adjusted by whether it was overloaded or
+    underloaded in the batch; "The DeepSeekMoE Architecture.", configuration
+    table: "aux-loss-free bias"). Reading (the pages give the direction only):
+    overloaded = more than the mean load T*k/N pairs, which lowers b_e by
+    gamma; underloaded raises it by gamma; exactly the mean leaves it.
+    Returns fp64; the caller's bias is fp32, so compare after rounding."""
+    counts = np.asarray(counts, dtype=np.int64)
+    N = counts.shape[0]
+    mean = T * k / N  # exact comparison below uses integers
+    direction = np.sign(T * k - N * counts)  # +1 under, -1 over, 0 at the mean
+    assert np.all((counts > mean) == (direction < 0))
+    return np.asarray(b, dtype=np.float64) + gamma * direction
+
+
 # ---------------------------------------------------------------- experts ----
 
 def expert_ffn(x: np.ndarray, W1: np.ndarray, W3: np.ndarray, W2: np.ndarray) -> np.ndarray:

@@ -117,4 +117,9 @@ def test_argument_errors_need_no_device(L):
     # shared weights required when n_shared > 0
     assert L.moe_forward(ctypes.byref(cfg), 4, fake, fake, None, fake, fake, fake, None, None, None, fake,
                          None, None, fake, 1 << 40, None) == 1
+    # bias update: null / misaligned pointers, non-finite rate
+    assert L.moe_bias_update(ctypes.byref(cfg), 4, None, ctypes.c_float(1e-3), fake, None) == 1
+    assert L.moe_bias_update(ctypes.byref(cfg), 4, fake, ctypes.c_float(1e-3), fake + 2, None) == 1
+    assert L.moe_bias_update(ctypes.byref(cfg), 4, fake, ctypes.c_float(float("nan")), fake, None) == 1
+    assert L.moe_bias_update(None, 4, fake, ctypes.c_float(1e-3), fake, None) == 1
     assert L.moe_last_cuda_error() == 0

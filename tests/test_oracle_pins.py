@@ -358,3 +358,30 @@ def test_permutation_against_sorted_pairs():
     assert [t * k + s for (_, t, s) in pairs] == perm.tolist()
     assert counts.tolist() == [sum(1 for p in pairs if p[0] == e) for e in range(N)]
     assert offsets[0] == 0 and offsets[-1] == T * k
+
+
+# --------------------------------------------------- bias update (balancing) --
+
+def test_bias_update_hand_example():
+    # N = 4 experts, T = 6 tokens, k = 2: mean load 3 pairs per expert.
+    # counts 5 (over), 3 (at the mean), 2 and 2 (under) -> -g, 0, +g, +g
+    b = np.array([0.25, -0.5, 0.0, 1.0])
+    got = oracle.bias_update(b, np.array([5, 3, 2, 2]), T=6, k=2, gamma=0.125)
+    assert np.array_equal(got, [0.125, -0.5, 0.125, 1.125])
+
+
+def test_bias_update_properties():
+    rng = np.random.default_rng(7)
+    for _ in range(20):
+        N, T, k = 16, int(rng.integers(1, 64)), int(rng.integers(1, 5))
+        # a random assignment of T*k pairs to experts
+        counts = np.bincount(rng.integers(0, N, size=T * k), minlength=N)
+        b = rng.normal(size=N)
+        new = oracle.bias_update(b, counts, T, k, 1e-3)
+        step = new - b
+        mean = T * k / N
+        assert np.all(step[counts > mean] < 0) and np.all(step[counts < mean] > 0)
+        assert np.all(step[counts == mean] == 0)
+        assert np.allclose(np.abs(step[counts != mean]), 1e-3)
+    # a perfectly balanced batch leaves the bias alone
+    assert np.array_equal(oracle.bias_update(np.ones(8), np.full(8, 3), T=12, k=2, gamma=0.5), np.ones(8))

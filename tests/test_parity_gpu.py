@@ -131,6 +131,30 @@ def test_route_matches_forward_routing_and_is_deterministic():
     assert (gi.cpu().numpy() == i1).all() and (gg.cpu().numpy() == g1).all()
 
 
+def test_bias_update_bit_exact():
+    # counts straight from the GPU's own routing and dispatch, plus a crafted
+    # vector with loads at, above and below the mean
+    s = SMALL["v3_like_small"]
+    cfg = cfg_of(s)
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    _, gidx, _ = run_forward(s, w, x)
+    ws = workspace(cfg, s.T)
+    counts = torch.zeros(s.n_routed, dtype=torch.int32, device="cuda")
+    moe.dispatch(cfg, s.T, torch.from_numpy(gidx).cuda(), counts, None, None, ws)
+    crafted = np.zeros(s.n_routed, dtype=np.int32)
+    mean = s.T * s.top_k // s.n_routed
+    crafted[: s.n_routed // 2] = mean
+    crafted[s.n_routed // 2:] = mean + np.arange(s.n_routed - s.n_routed // 2) % 3 - 1
+    for c in (counts, torch.from_numpy(crafted).cuda()):
+        b0 = torch.from_numpy(np.random.default_rng(3).normal(size=s.n_routed).astype(np.float32)).cuda()
+        b = b0.clone()
+        moe.bias_update(cfg, s.T, c, 1e-3, b)
+        torch.cuda.synchronize()
+        ref = oracle.bias_update(b0.cpu().numpy(), c.cpu().numpy(), s.T, s.top_k, np.float64(np.float32(1e-3)))
+        assert np.array_equal(b.cpu().numpy(), ref.astype(np.float32))
+
+
 def test_identical_experts_invariant():
     # every routed expert identical, normalised gates: y = 2.5 FFN(x) + shared(x) whatever the routing
     s = SMALL["v3_like_small"]
@@ -181,10 +205,10 @@ def test_abi_errors_on_device_buffers():
 # ------------------------------------------------------------- full size ----
 
 SAMPLES = {"gshard_tiny_f32": None, "dsmoe_2b_bf16": 64, "v2_layer_bf16": 16, "v3_prefill_bf16": 16,
-           "v3_decode_bf16": None, "v3_prefill_t16k_bf16": 16}
+           "v3_decode_bf16": None, "v3_prefill_t16k_bf16": 16, "v2_device_limited_bf16": 16}
 
 
-@pytest.mark.parametrize("name", mi.ORDER + ["v3_prefill_t16k_bf16"])
+@pytest.mark.parametrize("name", mi.ORDER + ["v3_prefill_t16k_bf16", "v2_device_limited_bf16"])
 def test_full_size_config(name):
     s = mi.SHAPES[name]
     w = mdev.device_all(s)
