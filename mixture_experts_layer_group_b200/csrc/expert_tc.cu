@@ -145,13 +145,17 @@ MOE_DEV Unit decode_unit(const TcParams& p, int u) {
   }
   const int local = u - __ldg(p.unit_base + lo);
   const int rows = __ldg(p.grp_rows + lo);
+  // a group's rows split into nc chunks of (almost) equal size, so the
+  // chunks that share a weight tile run at the same pace and keep reading
+  // its lines from L2 together
   const int nc = (rows + kMaxTok - 1) / kMaxTok;
+  const int cs = (rows + nc - 1) / nc;
   Unit un;
   un.g = lo;
   un.f = local / nc;
-  un.tok0 = (local % nc) * kMaxTok;
+  un.tok0 = (local % nc) * cs;
   const int left = rows - un.tok0;
-  un.ntok = left < kMaxTok ? left : kMaxTok;
+  un.ntok = left < cs ? left : cs;
   un.nchunks = nc;
   return un;
 }
