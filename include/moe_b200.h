@@ -171,6 +171,12 @@ MOE_API moe_status moe_forward(const moe_cfg* cfg, int64_t T, const void* x, con
  * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous; the
  * caller synchronises the stream before reading y_host. Weights stay in
  * device memory. Needs moe_workspace_size_host() bytes of workspace.
+ * The host-to-device copy runs on a copy stream the library keeps for the
+ * workspace (with two events; created on first use, kept until the process
+ * exits) and waits only until the previous call on the same workspace has
+ * finished reading its staged x, so back-to-back calls overlap one call's
+ * input copy with the previous call's down projection and output copy. The
+ * output copy stays on `stream`.
  */
 MOE_API moe_status moe_workspace_size_host(const moe_cfg* cfg, int64_t T, size_t* bytes);
 MOE_API moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,

@@ -705,7 +705,7 @@ cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStream_t s,
-                                   cudaEvent_t between) {
+                                   cudaEvent_t between, cudaEvent_t between2) {
   const int sms = device_sm_count();
   cudaError_t err0 = cudaMemsetAsync(a.sched, 0, 2 * sizeof(int), s);
   if (err0 != cudaSuccess) return err0;
@@ -744,6 +744,7 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   const int64_t units1 = chunks_bound * ((max_cols1 + kTcBN1 - 1) / kTcBN1);
   cudaError_t err = launch_one<kSwiGLU>(g1, (int)(units1 < sms ? units1 : sms), s);
   if (err == cudaSuccess && between) err = cudaEventRecord(between, s);
+  if (err == cudaSuccess && between2) err = cudaEventRecord(between2, s);
   if (err != cudaSuccess) return err;
 
   TcParams g2{};

@@ -116,12 +116,13 @@ struct GemmArgs {
 };
 
 // Tensor-core (bf16) expert GEMMs: SwiGLU projection then gated down
-// projection; `between` (optional) is recorded on s between the two launches.
+// projection; `between` and `between2` (optional) are recorded on s between
+// the two launches.
 cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStream_t s,
-                                   cudaEvent_t between);
+                                   cudaEvent_t between, cudaEvent_t between2 = nullptr);
 // fp32 SIMT expert GEMMs.
 cudaError_t launch_expert_gemms_simt(const Problem& p, const GemmArgs& a, cudaStream_t s,
-                                     cudaEvent_t between);
+                                     cudaEvent_t between, cudaEvent_t between2 = nullptr);
 
 // y[t] = sum over the token's rows slot_pos[t, 0..k) (ascending expert) of
 // y_rows, plus the shared row y_rows[R + t]

@@ -3,6 +3,8 @@
 //   router -> dispatch -> gather -> SwiGLU GEMM -> gate GEMM -> combine,
 // all on the caller's stream with no host synchronisation.
 #include <cstring>
+#include <mutex>
+#include <unordered_map>
 
 #include "common.cuh"
 #include "internal.h"
@@ -166,7 +168,8 @@ DispatchBuffers dispatch_buffers(const Layout& L, void* ws, const int32_t* idx, 
 moe_status forward_device(const Problem& p, const Layout& L, const void* x, const void* W_r,
                           const float* b, const void* W1, const void* W3, const void* W2,
                           const void* Ws1, const void* Ws3, const void* Ws2, void* y,
-                          int32_t* idx_out, float* gates_out, void* ws, cudaStream_t s) {
+                          int32_t* idx_out, float* gates_out, void* ws, cudaStream_t s,
+                          cudaEvent_t x_released = nullptr) {
   int32_t* idx = at<int32_t>(ws, L.idx);
   float* gates = at<float>(ws, L.gates);
   cudaError_t e0 = cudaMemsetAsync(at<void>(ws, L.status), 0, 4, s);
@@ -203,8 +206,9 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
   ga.gate_perm = db.gate_perm;
   ga.status = db.status;
   ga.sched = at<int>(ws, L.sched);
-  e = tc ? launch_expert_gemms_tc(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr)
-         : launch_expert_gemms_simt(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr);
+  // x is not read after the SwiGLU GEMM: x_released (optional) marks that point
+  e = tc ? launch_expert_gemms_tc(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr, x_released)
+         : launch_expert_gemms_simt(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr, x_released);
   if (e == cudaSuccess) e = mark_stage(5, s);
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch_combine(p, ga.y_rows, db.slot_pos, y, s);
@@ -219,6 +223,43 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return MOE_OK;
+}
+
+// Per-workspace state of moe_forward_host: a non-blocking copy stream and
+// two events (no device memory), created on first use and kept for the
+// process lifetime.
+struct HostPipe {
+  int device = -1;
+  cudaStream_t copy = nullptr;
+  cudaEvent_t x_ready = nullptr;  // the staged x has landed
+  cudaEvent_t x_free = nullptr;   // the last call on this workspace no longer reads it
+  bool pending = false;           // x_free has been recorded
+};
+std::mutex g_pipe_mu;
+std::unordered_map<const void*, HostPipe> g_pipes;
+
+cudaError_t host_pipe(const void* ws, HostPipe** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe& hp = g_pipes[ws];
+  if (hp.device != dev) {
+    if (hp.copy) {  // a different device reuses this address: start over
+      cudaStreamDestroy(hp.copy);
+      cudaEventDestroy(hp.x_ready);
+      cudaEventDestroy(hp.x_free);
+      hp = HostPipe{};
+    }
+    e = cudaStreamCreateWithFlags(&hp.copy, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.x_ready, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.x_free, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+    hp.device = dev;
+    hp.pending = false;
+  }
+  *out = &hp;
+  return cudaSuccess;
 }
 
 moe_status check_weights(const Problem& p, const void* W_r, const float* b, const void* W1,
@@ -330,10 +371,20 @@ moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, c
   const size_t bytes = (size_t)p.T * p.d * p.elem;
   void* xd = at<void>(ws, L.x_stage);
   void* yd = at<void>(ws, L.y_stage);
-  cudaError_t e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s);
+  // The host-to-device copy runs on the workspace's own copy stream, after
+  // the previous call on this workspace released the staged x (end of its
+  // SwiGLU GEMM): consecutive calls overlap this copy with the previous
+  // call's down projection, combine and device-to-host copy.
+  HostPipe* hp = nullptr;
+  cudaError_t e = host_pipe(ws, &hp);
+  if (e == cudaSuccess && hp->pending) e = cudaStreamWaitEvent(hp->copy, hp->x_free, 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, hp->copy);
+  if (e == cudaSuccess) e = cudaEventRecord(hp->x_ready, hp->copy);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->x_ready, 0);
   if (e != cudaSuccess) return cuda_fail(e);
-  st = forward_device(p, L, xd, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, yd, nullptr, nullptr, ws, s);
+  st = forward_device(p, L, xd, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, yd, nullptr, nullptr, ws, s, hp->x_free);
   if (st != MOE_OK) return st;
+  hp->pending = true;
   e = cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return MOE_OK;

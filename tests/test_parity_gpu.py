@@ -185,6 +185,26 @@ def test_forward_host_matches_device_forward():
     assert torch.equal(yh, y_dev.cpu())
 
 
+def test_forward_host_back_to_back_calls():
+    # consecutive calls on one workspace overlap the next input copy with the
+    # previous call's tail: every call must still see its own tokens
+    s = SMALL["v3_like_small"]
+    w = mdev.device_all(s)
+    cfg = cfg_of(s)
+    ws = workspace(cfg, s.T, host=True)
+    wargs = (w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"])
+    xs = [mdev.device_tensor(s.with_(seed=s.seed + i), "x") for i in range(4)]
+    refs = [run_forward(s, w, x)[0].cpu() for x in xs]
+    xh = [x.cpu().pin_memory() for x in xs]
+    yh = [torch.empty_like(h).pin_memory() for h in xh]
+    for _ in range(2):
+        for i in range(4):  # no synchronisation between calls
+            moe.forward_host(cfg, s.T, xh[i], *wargs, yh[i], ws)
+        torch.cuda.synchronize()
+        for i in range(4):
+            assert torch.equal(yh[i], refs[i]), i
+
+
 def test_abi_errors_on_device_buffers():
     s = SMALL["v3_like_small"]
     cfg = cfg_of(s)
