@@ -248,6 +248,14 @@ MOE_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
                : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before its predecessor ends; griddep_wait blocks
+// until the predecessor grid has completed and its writes are visible (a
+// no-op without the attribute); griddep_launch_dependents lets the
+// dependent grid start once every CTA of this grid has called it or exited.
+MOE_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MOE_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 MOE_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 MOE_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 

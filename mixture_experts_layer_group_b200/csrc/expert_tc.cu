@@ -274,6 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
   if (warp == 0) {
     // ------------------------------------------------- scheduler + producer --
     if (lane == 0) {
+      // the down GEMM may start while the SwiGLU GEMM drains (programmatic
+      // launch): nothing it loads may be read before that grid has finished
+      if (MODE == kGateDown) griddep_wait();
       // a weight tile read by one unit only is streamed once: evict it first;
       // tiles shared by the chunks of a large group stay at normal priority
       const uint64_t pol_once = policy_evict_first();
@@ -337,7 +340,12 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           u = load_volatile(&sh.ring[q]);
           mbar_arrive_cluster(in_first(&sh.ring_empty[q]));
         }
-        if (u < 0) break;
+        if (u < 0) {
+          // no units left for this CTA: the down GEMM may start on SMs as
+          // they free up
+          if (MODE == kSwiGLU) griddep_launch_dependents();
+          break;
+        }
         const Unit un = decode_unit(p, u);
         const bool shared = un.g == p.N;
         const int K = shared ? p.k_shared : p.k_routed;
@@ -669,17 +677,19 @@ bool make_store_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
 }
 
 template <int MODE>
-cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s) {
+cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s, bool programmatic) {
   static int configured_device = -1;
   static int max_clusters = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;
@@ -699,6 +709,7 @@ cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s) {
   int clusters = max_clusters;
   if (max_units < clusters) clusters = max_units > 0 ? max_units : 1;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.numAttrs = programmatic ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, expert_gemm_tc_kernel<MODE>, prm);
 }
 
@@ -742,7 +753,7 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g1.status = a.status;
   const int64_t max_cols1 = p.F > p.nsF ? p.F : p.nsF;
   const int64_t units1 = chunks_bound * ((max_cols1 + kTcBN1 - 1) / kTcBN1);
-  cudaError_t err = launch_one<kSwiGLU>(g1, (int)(units1 < sms ? units1 : sms), s);
+  cudaError_t err = launch_one<kSwiGLU>(g1, (int)(units1 < sms ? units1 : sms), s, false);
   if (err == cudaSuccess && between) err = cudaEventRecord(between, s);
   if (err == cudaSuccess && between2) err = cudaEventRecord(between2, s);
   if (err != cudaSuccess) return err;
@@ -774,7 +785,9 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g2.gate_perm = a.gate_perm;
   g2.status = a.status;
   const int64_t units2 = chunks_bound * ((p.d + kTcBN2 - 1) / kTcBN2);
-  return launch_one<kGateDown>(g2, (int)(units2 < sms ? units2 : sms), s);
+  // the down GEMM overlaps the SwiGLU GEMM's drain unless an event must be
+  // recorded between the two
+  return launch_one<kGateDown>(g2, (int)(units2 < sms ? units2 : sms), s, !between && !between2);
 }
 
 }  // namespace moe
