@@ -311,55 +311,97 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
-def oracle_sample_time(s: mi.LayerShape, n_tok: int, seed: int):
-    """Times the fp64 oracle on n_tok sampled tokens of the workload (the
-    weights those tokens need are generated in their storage dtype first;
-    widening to fp64 and all arithmetic are inside the timed call)."""
+def cpu_baseline(s: mi.LayerShape, n_tok: int):
+    """The oracle, as it stands, on the host cores: the layer forward for a
+    resident sample of n_tok tokens, repeated for about 10 s of CPU work."""
+    sample = reference_sample(s, sample_token_cap(s, n_tok), 1234)
+    n = sample[0].shape[0]
+    times = [oracle_step(sample)]
+    while sum(times) < 10.0 and len(times) < 200:
+        times.append(oracle_step(sample))
+    dt = float(np.mean(times))
+    return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{n} seeded tokens of {s.name} (router, their experts, shared MLP, combine), fp64 numpy "
+                      f"oracle with resident fp64 weights, {len(times)} repetitions, {sum(times):.1f} s"}
+
+
+def reference_sample(s: mi.LayerShape, n_tok: int, seed: int):
+    """The reference arm's resident inputs: n_tok seeded tokens of the
+    workload with the router and the weights of every expert they use,
+    widened to the oracle's fp64 once (as the GPU arm's weights sit in HBM
+    before its timed region)."""
     import oracle
     rows = np.sort(np.random.default_rng(seed).choice(s.T, n_tok, replace=False))
-    x64 = mi.bf16_to_f32(mi.host_rows(s, "x", rows)).astype(np.float64) if s.dtype == "bf16" else \
-        mi.host_rows(s, "x", rows).astype(np.float64)
-    W_r = mi.host_tensor(s, "W_r").reshape(s.n_routed, s.d)
+    widen = (lambda a: mi.bf16_to_f32(a).astype(np.float64)) if s.dtype == "bf16" else \
+        (lambda a: a.astype(np.float64))
+    x64 = widen(mi.host_rows(s, "x", rows))
+    W_r = widen(mi.host_tensor(s, "W_r").reshape(s.n_routed, s.d))
     b = mi.host_tensor(s, "b").astype(np.float64) if s.bias else None
     rcfg = oracle.RouterCfg(n_routed=s.n_routed, top_k=s.top_k, score=s.score, n_groups=s.n_groups,
                             topk_groups=s.topk_groups, normalize=s.normalize, route_scale=s.route_scale,
                             group_score=s.group_score)
-    widen = (lambda a: mi.bf16_to_f32(a).astype(np.float64)) if s.dtype == "bf16" else \
-        (lambda a: a.astype(np.float64))
-    r = oracle.route(x64, widen(W_r), b, rcfg)
-    need = sorted(set(r.idx.reshape(-1).tolist()))
-    stored = {e: mi.host_expert(s, e) for e in need}
+    need = sorted(set(oracle.route(x64, W_r, b, rcfg).idx.reshape(-1).tolist()))
+    experts = {e: tuple(widen(a) for a in mi.host_expert(s, e)) for e in need}
     shared = mi.host_shared(s)
+    shared = None if shared is None else tuple(widen(a) for a in shared)
+    return x64, W_r, b, rcfg, experts, shared
+
+
+def oracle_step(sample) -> float:
+    """Seconds for one oracle layer forward over a resident sample."""
+    import oracle
+    x64, W_r, b, rcfg, experts, shared = sample
     t0 = time.perf_counter()
-    oracle.forward(x64, widen(W_r), b, rcfg, lambda e: tuple(widen(a) for a in stored[e]),
-                   None if shared is None else tuple(widen(a) for a in shared))
+    oracle.forward(x64, W_r, b, rcfg, lambda e: experts[e], shared)
     return time.perf_counter() - t0
 
 
-def cpu_baseline(s: mi.LayerShape, n_tok: int):
-    dt = oracle_sample_time(s, n_tok, 1234)
-    return {"value": round(n_tok / dt, 3), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"{n_tok} sampled tokens of {s.name} (all their experts + shared), fp64 numpy oracle, "
-                      f"{dt:.1f} s"}
+def sample_token_cap(s: mi.LayerShape, want: int) -> int:
+    """At most `want` tokens, fewer if their fp64 expert weights would take
+    more than a quarter of the host's available memory."""
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:  # no psutil: trust the request
+        return want
+    per_expert = 3 * s.d * s.d_ff * 8
+    n = want
+    while n > 1 and (n * s.top_k + s.n_shared) * per_expert > avail // 4:
+        n -= 1
+    return n
 
 
 def run_reference(args, rank, world):
+    """The reference arm of this tier: the fp64 oracle, as it stands, on the
+    host cores. Each step runs the whole layer forward (router, every chosen
+    expert, shared MLP, combine) for the same sample of tokens; the sample
+    (1 to 4 tokens) is sized from a first timing so the run stays within
+    about two minutes."""
     if rank != 0:
         return None
     s = mi.SHAPES[args.config]
     from moe_inputs import build as gen_build
     gen_build.build_host()
+
+    step = oracle_step
+    probe = reference_sample(s, 1, 99)
+    t1 = min(step(probe) for _ in range(2))
+    n_tok = int(max(1, min(sample_token_cap(s, args.cpu_tokens),
+                           120.0 / max(1e-9, (args.steps + args.warmup) * t1))))
+    sample = probe if n_tok == 1 else reference_sample(s, n_tok, 99)
     for _ in range(args.warmup):
-        oracle_sample_time(s, args.cpu_tokens, 99)
-    times = [oracle_sample_time(s, args.cpu_tokens, 100 + k) for k in range(args.steps)]
+        step(sample)
+    times = [step(sample) for _ in range(args.steps)]
     ms = 1e3 * float(np.mean(times))
-    v = args.cpu_tokens / (ms / 1e3)
+    v = n_tok / (ms / 1e3)
+    desc = (f"{n_tok} seeded token(s) of {s.name} per step, the layer forward for them (router, their "
+            f"experts, shared MLP, combine) in the fp64 numpy oracle, weights resident in fp64")
     return {"metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": describe(s), "global_batch": args.cpu_tokens},
+            "config": {"workload": describe(s), "global_batch": n_tok},
             "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
-                             "sample": f"{args.cpu_tokens} sampled tokens per step of {s.name}"},
+                             "sample": desc},
             "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
