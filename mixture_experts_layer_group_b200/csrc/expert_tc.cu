@@ -51,6 +51,8 @@
 // MOE_DEV_WAIT_TIMEOUT, drains its own copies and MMAs (bounded again),
 // frees its tensor memory and exits.
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -678,10 +680,13 @@ bool make_store_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
 
 template <int MODE>
 cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s, bool programmatic) {
-  static int configured_device = -1;
-  static int max_clusters = 0;
+  // per device: the shared-memory opt-in done and the resident cluster count
+  static std::mutex mu;
+  static int max_clusters_of[kMaxDevices] = {};
   int dev = 0;
-  cudaGetDevice(&dev);
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 != cudaSuccess) return e0;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -695,18 +700,21 @@ cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s, bool 
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(expert_gemm_tc_kernel<MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
-    int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, expert_gemm_tc_kernel<MODE>, &cfg);
-    if (e != cudaSuccess) return e;
-    max_clusters = n > 0 ? n : 1;
-    configured_device = dev;
+  int clusters = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (max_clusters_of[dev] == 0) {
+      cudaError_t e = cudaFuncSetAttribute(expert_gemm_tc_kernel<MODE>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      if (e != cudaSuccess) return e;
+      cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, expert_gemm_tc_kernel<MODE>, &cfg);
+      if (e != cudaSuccess) return e;
+      max_clusters_of[dev] = n > 0 ? n : 1;
+    }
+    clusters = max_clusters_of[dev];
   }
-  int clusters = max_clusters;
   if (max_units < clusters) clusters = max_units > 0 ? max_units : 1;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.numAttrs = programmatic ? 2 : 1;

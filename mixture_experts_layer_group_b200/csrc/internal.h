@@ -24,6 +24,7 @@ constexpr int kSimtBN = 64;
 constexpr int kChunkTokens = 32;  // dispatch: tokens per warp chunk
 constexpr int kMaxRouted = 512;
 constexpr int kMaxTopK = 16;
+constexpr int kMaxDevices = 64;   // devices a process may use the library on
 
 struct Problem {
   int64_t T;

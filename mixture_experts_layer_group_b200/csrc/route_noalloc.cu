@@ -19,7 +19,6 @@ namespace {
 // Largest scratch a call may use: the router's fp32 logits, T * n_routed * 4
 // bytes (the router splits its reduction only as far as the array allows).
 constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB
-constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_route_scratch[kNoallocScratchBytes];
 

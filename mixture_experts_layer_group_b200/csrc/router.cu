@@ -12,6 +12,7 @@
 // result stays deterministic.
 #include <cfloat>
 #include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -389,18 +390,23 @@ cudaError_t launch_router(const Problem& p, const void* x, const void* W_r, cons
   if (S < 1) return cudaErrorInvalidValue;
   const int k_len = ((p.d + S - 1) / S + kLBK - 1) / kLBK * kLBK;
   dim3 grid((unsigned)((p.N + kLBN - 1) / kLBN), (unsigned)((p.T + kLBT - 1) / kLBT), (unsigned)S);
-  static int configured_device = -1;
+  static std::mutex mu;
+  static bool configured[kMaxDevices] = {};  // shared-memory opt-in done, per device
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (configured_device != dev) {
-    err = cudaFuncSetAttribute(router_logits_kernel<__nv_bfloat16>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, kLSmemBytes);
-    if (err == cudaSuccess)
-      err = cudaFuncSetAttribute(router_logits_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kLSmemBytes);
-    if (err != cudaSuccess) return err;
-    configured_device = dev;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured[dev]) {
+      err = cudaFuncSetAttribute(router_logits_kernel<__nv_bfloat16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kLSmemBytes);
+      if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(router_logits_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   kLSmemBytes);
+      if (err != cudaSuccess) return err;
+      configured[dev] = true;
+    }
   }
   if (p.dtype == MOE_BF16)
     router_logits_kernel<__nv_bfloat16><<<grid, kLThreads, kLSmemBytes, s>>>(

@@ -33,6 +33,13 @@ SMALL = {
     "tiny_f32": LS("tiny_f32", T=77, d=136, n_routed=12, n_shared=1, d_ff=200, top_k=3, score="sigmoid",
                    normalize=True, route_scale=2.5, dtype="f32", seed=15, bias=True),
     "gshard_tiny_f32": mi.SHAPES["gshard_tiny_f32"],
+    # the library's limits: 512 routed experts, top-16, 32 groups
+    "max_limits": LS("max_limits", T=300, d=256, n_routed=512, n_shared=1, d_ff=128, top_k=16,
+                     score="sigmoid", n_groups=32, topk_groups=8, normalize=True, route_scale=2.5, seed=16,
+                     bias=True),
+    # bf16 with reduction lengths that are not multiples of the 64-wide K block
+    "bf16_ragged_k": LS("bf16_ragged_k", T=97, d=200, n_routed=10, n_shared=1, d_ff=136, top_k=3,
+                        score="softmax", seed=17),
 }
 
 
