@@ -30,6 +30,13 @@ Readings where the pages are silent (each is listed in the design notes):
     (TG+1)-th group score); slot-order ties are flagged separately.
   * the residual is not part of Delta_ffn.
 No value is rounded: inputs are widened exactly to fp64 and stay there.
+
+Pins (tests/test_oracle_pins.py): selection by brute force over all subsets,
+the printed parameter and combination counts, closed forms, and identities
+(segmentation, shared fusion, dense ceiling, identical experts, GShard
+special case). The pages print no worked layer output, so output values are
+pinned only through those identities and closed forms: beyond them, parity
+unpinned.
 """
 from __future__ import annotations
 
