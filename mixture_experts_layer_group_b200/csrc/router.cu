@@ -290,14 +290,15 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
   if (a.G > 1) {
     // group scores: lane g keeps the score of group g (G <= 32)
     const int S = N / a.G;
+    int grp[V];  // group of each of this lane's experts
+#pragma unroll
+    for (int j = 0; j < V; ++j) grp[j] = (32 * j + lane) / S;
     float my_gs = -INFINITY;
     for (int g = 0; g < a.G; ++g) {
       float t1 = -INFINITY, t2 = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < V; ++j) {
-        int e = 32 * j + lane;
-        if (e < N && e / S == g) merge_top2(t1, t2, key[j], -INFINITY);
-      }
+      for (int j = 0; j < V; ++j)
+        if (32 * j + lane < N && grp[j] == g) merge_top2(t1, t2, key[j], -INFINITY);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
         float o1 = __shfl_xor_sync(0xffffffffu, t1, off);
@@ -314,10 +315,8 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
       if (lane == c.e) my_gs = -INFINITY;
     }
 #pragma unroll
-    for (int j = 0; j < V; ++j) {
-      int e = 32 * j + lane;
-      if (e < N && !((allowed >> (e / S)) & 1u)) key[j] = -INFINITY;
-    }
+    for (int j = 0; j < V; ++j)
+      if (32 * j + lane < N && !((allowed >> grp[j]) & 1u)) key[j] = -INFINITY;
   }
 
   int sel_e = 0;
