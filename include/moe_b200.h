@@ -92,7 +92,8 @@ enum {
  *   route_scale  gate multiplier (2.5 for the DeepSeek-V3 layer, 1 for GShard)
  *   group_score  how a group is scored for the group limit: the sum of its
  *                two largest s+b (MOE_GROUP_TOP2_SUM) or its largest (MOE_GROUP_MAX)
- *   dtype        MOE_F32 (SIMT fp32 path) or MOE_BF16 (tensor-core path)
+ *   dtype        MOE_F32 (SIMT fp32 path) or MOE_BF16 (tensor-core expert GEMMs; the
+ *                router runs on the FP32 pipes for both)
  */
 typedef struct moe_cfg {
   int32_t d;
