@@ -6,8 +6,8 @@
 // 16, at most 256, half of them in each CTA), so each SM streams its own
 // weight rows but only half of the token rows, and the MMA work follows the
 // real number of tokens per expert instead of a padded row tile. A unit
-// issues two pair MMAs per K step on one shared token tile. Two launches per
-// layer:
+// issues two pair MMAs (its two 128-row A halves per CTA) per K step on one
+// shared token tile. Two launches per layer:
 //
 //   SwiGLU GEMM  unit = (group, 256 features, <= 256 tokens): CTA r holds
 //                features 128 r .. 128 r + 127 of the unit; half 0 of its
@@ -23,29 +23,34 @@
 //
 // Groups 0..N-1 are the routed experts over their expert-contiguous token
 // rows; group N is the fused shared MLP over all T tokens, in the same
-// persistent launch. Units of one group are consecutive, weight-tile major
-// and token-chunk minor. The pair's first CTA takes units from a global
-// counter, so the chunks that share a weight tile start together (they read
-// it once through L2) and the last units balance across SMs.
+// persistent launch. A group of more than 256 rows is cut into equal chunks.
+// Units of one group are consecutive, weight-tile major and token-chunk
+// minor. The pair's first CTA takes units from a global counter, so the
+// chunks that share a weight tile start together (they read it once through
+// L2) and the last units balance across SMs. The gate GEMM is launched with
+// programmatic stream serialization and waits for the SwiGLU grid before its
+// first load.
 //
 // CTA roles (320 threads, one CTA per SM, persistent; the same roles in both
 // CTAs of a pair except the MMA issuer, which only the first CTA has):
 //   warp 0      TMA producer (one lane). In CTA 0 it also takes unit ids and
 //               hands them to both CTAs through shared-memory rings. Stages
-//               are variable-size pieces (32 KB of weights + one token box of
-//               32, 64 or 128 rows, 4 / 8 / 16 KB) of a 208 KB byte ring; the bytes of both CTAs complete
-//               on CTA 0's stage barrier; weights read by one unit only are
-//               evict-first
+//               are variable-size pieces of a 208 KB byte ring: per 64-wide
+//               K block, 32 KB of weights (two 128-row boxes) and one token
+//               box of 32, 64 or 128 rows (4 / 8 / 16 KB; the TMA engine's
+//               cost is per box); the bytes of both CTAs complete on CTA 0's
+//               stage barrier; weights read by one unit only are evict-first
 //   warp 1      TMEM owner (both CTAs, pair allocation) + UMMA issuer (CTA 0,
 //               one lane): 2 x 4 pair MMAs (256 x N x 16) per stage. Each
 //               CTA's TMEM holds two buffers of 2 x 128 fp32 columns: a unit
 //               of <= 128 tokens takes one buffer (the next unit's MMAs
 //               overlap its epilogue), a larger unit takes both (2 x 256)
 //   warps 2..9  epilogue, two warps per TMEM lane quadrant taking turns on
-//               32-token blocks: each warp reads its quadrant, applies SwiGLU
-//               or the gate, transposes the 32 x 32 block through its own
-//               shared-memory tile (bf16) and writes it with
-//               one TMA tensor store (a ragged last block with 64-byte row
+//               32-token blocks: each warp reads its quadrant in the m16n8
+//               layout (tcgen05.ld 16x256b), applies SwiGLU or the gate,
+//               transposes the 32 x 32 block into its own 64-byte-swizzled
+//               shared-memory tile with stmatrix.trans and writes it with one
+//               TMA tensor store (a ragged last block with 64-byte row
 //               stores); no barrier between epilogue warps per block
 // Every mbarrier wait is bounded; on a timeout a CTA records
 // MOE_DEV_WAIT_TIMEOUT, drains its own copies and MMAs (bounded again),
