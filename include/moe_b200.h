@@ -252,6 +252,18 @@ MOE_API moe_status moe_route_noalloc(const moe_cfg* cfg, int64_t T, const void* 
 MOE_API moe_status moe_bias_update(const moe_cfg* cfg, int64_t T, const int32_t* counts, float gamma, float* b,
                                    void* stream);
 
+/*
+ * Self-check of the failure path (no counterpart in the pages): launches a
+ * one-warp kernel that waits, with the same bounded wait every pipeline in
+ * the library uses, on a barrier that nothing ever completes. After the wait
+ * limit (1 s) the kernel records MOE_DEV_WAIT_TIMEOUT and returns; the call
+ * synchronises `stream` and writes the recorded bits to *bits (expected:
+ * MOE_DEV_WAIT_TIMEOUT). The CUDA context stays usable. Takes about 1 s.
+ * Errors: MOE_ERR_INVALID_ARG for a null bits; MOE_ERR_CUDA for a failed
+ * launch or copy.
+ */
+MOE_API moe_status moe_selftest_wait_timeout(uint32_t* bits, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 MOE_API const char* moe_status_string(moe_status status);
 

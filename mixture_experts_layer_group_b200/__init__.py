@@ -22,7 +22,7 @@ MOE_DEV_WAIT_TIMEOUT, MOE_DEV_BAD_EXPERT, MOE_DEV_DUP_EXPERT, MOE_DEV_TMEM_ALLOC
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE"}
 EXPORTS = ["moe_workspace_size", "moe_workspace_size_host", "moe_route", "moe_dispatch", "moe_forward",
-           "moe_forward_host", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update",
+           "moe_forward_host", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update", "moe_selftest_wait_timeout",
            "moe_status_string", "moe_last_cuda_error"]
 STAGES = ["router", "dispatch", "gather", "gemm_swiglu", "gemm_gate", "combine"]
 
@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
         L.moe_route_noalloc.argtypes = [CFG, I64, P, P, P, P, P, P]
         L.moe_bias_update.argtypes = [CFG, I64, P, ctypes.c_float, P, P]
+        L.moe_selftest_wait_timeout.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_last_cuda_error.argtypes = []
@@ -142,6 +143,14 @@ def bias_update(cfg, T, counts, gamma, b, stream=None):
     the mean load T * top_k / N, += gamma where it falls short (in place)."""
     _check("moe_bias_update", lib().moe_bias_update(ctypes.byref(cfg), T, _ptr(counts), float(gamma), _ptr(b),
                                                     _stream(stream)))
+
+
+def selftest_wait_timeout(stream=None) -> int:
+    """Runs the bounded-wait self-check (about 1 s) and returns the device
+    status bits it recorded (MOE_DEV_WAIT_TIMEOUT when the wait gave up)."""
+    bits = ctypes.c_uint32(0)
+    _check("moe_selftest_wait_timeout", lib().moe_selftest_wait_timeout(ctypes.byref(bits), _stream(stream)))
+    return bits.value
 
 
 def dispatch(cfg, T, topk_idx, counts, offsets, perm, ws, ws_bytes=None, stream=None):

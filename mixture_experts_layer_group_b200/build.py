@@ -10,7 +10,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe_b200.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 SOURCES = ["moe_abi.cu", "router.cu", "tensor_map.cu", "dispatch.cu", "combine.cu", "expert_tc.cu", "expert_simt.cu",
-           "route_noalloc.cu", "bias_update.cu"]
+           "route_noalloc.cu", "bias_update.cu", "selftest.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
 

@@ -3,6 +3,8 @@
 Small layers (full oracle, several tiles and ragged tails) and the five
 layer configurations at full size (oracle on sampled tokens; routing on all
 tokens). Inputs come from the seeded generator on both sides."""
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -160,6 +162,16 @@ def test_bias_update_bit_exact():
         torch.cuda.synchronize()
         ref = oracle.bias_update(b0.cpu().numpy(), c.cpu().numpy(), s.T, s.top_k, np.float64(np.float32(1e-3)))
         assert np.array_equal(b.cpu().numpy(), ref.astype(np.float32))
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    # a wait that nothing completes runs out after the limit and is reported
+    # as a device-status bit; the same process then runs a layer correctly
+    t0 = time.perf_counter()
+    bits = moe.selftest_wait_timeout()
+    dt = time.perf_counter() - t0
+    assert bits == moe.MOE_DEV_WAIT_TIMEOUT and 0.9 < dt < 30.0, (bits, dt)
+    full_oracle_check(SMALL["single_token"])
 
 
 def test_identical_experts_invariant():
