@@ -164,6 +164,31 @@ def test_bias_update_bit_exact():
         assert np.array_equal(b.cpu().numpy(), ref.astype(np.float32))
 
 
+def test_forward_replays_from_a_cuda_graph():
+    # moe_forward issues only stream-ordered work (memsets, kernel launches),
+    # so a captured step replays to the same bits as an eager one
+    s = SMALL["v3_like_small"]
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    y_eager, _, _ = run_forward(s, w, x)
+    cfg = cfg_of(s)
+    ws = workspace(cfg, s.T)
+    y = torch.empty_like(x)
+    wargs = (w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"])
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        moe.forward(cfg, s.T, x, *wargs, y, ws, stream=side)  # per-device setup outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        moe.forward(cfg, s.T, x, *wargs, y, ws, stream=side)
+    y.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_eager)
+
+
 def test_bounded_wait_gives_up_and_context_survives():
     # a wait that nothing completes runs out after the limit and is reported
     # as a device-status bit; the same process then runs a layer correctly
