@@ -10,10 +10,8 @@ Everything here is written from the pages' statement of the layer:
     G_i = 2.5 s_i E_i / sum_j s_j E_j), the routed SwiGLU expert
     (g = x W1, u = x W3, a = g sigma(g), h = a * u, E = h W2), the shared
     expert, and Delta_ffn = y_routed + y_shared.
-  * the same page's quoted MoE.forward excerpt: tokens flattened to one axis,
-    fp32 (here fp64) accumulator, experts visited in ascending index, the
-    gate applied to the expert output, the shared MLP of width
-    n_shared * moe_inter_dim added to every token.
+  * the same page's quoted MoE module: tokens flattened to one axis, the
+    shared MLP of width n_shared * moe_inter_dim applied to every token.
   * "DeepSeekMoE" walkthrough, Step 2: the GShard router (dot product with
     every centroid, softmax over all of them, keep the top 2 values as gates,
     the rest are 0 -- no renormalisation).
@@ -226,36 +224,47 @@ def expert_ffn(x: np.ndarray, W1: np.ndarray, W3: np.ndarray, W2: np.ndarray) ->
     return h @ W2.T
 
 
+def gate_matrix(idx: np.ndarray, gates: np.ndarray, n_routed: int) -> np.ndarray:
+    """G [T, N]: G[t, i] is the gate of expert i for token t, zero for every
+    expert outside the token's selection (the equation list's G_i carries the
+    selection indicator E_sel_i, so unselected experts contribute nothing)."""
+    T, k = idx.shape
+    G = np.zeros((T, n_routed), dtype=np.float64)
+    rows = np.repeat(np.arange(T), k)
+    G[rows, idx.reshape(-1)] = gates.reshape(-1)
+    return G
+
+
 def forward(x: np.ndarray, W_r: np.ndarray, b, cfg: RouterCfg, expert, shared=None,
             routing: Routing | None = None, idx_override: np.ndarray | None = None):
-    """Delta_ffn = y_routed + y_shared for token rows x [T, d] (fp64).
+    """Delta_ffn = y_routed + y_shared for token rows x [T, d] (fp64), the
+    last steps of the "All 19 steps" list ("DeepSeek-V3.2-Exp · Mixture of
+    experts"): y_routed = sum_i G_i E_i(x) over the routed experts, with
+    E_i the SwiGLU expert and G_i zero outside the selection, and y_shared
+    the always-on shared MLP, ungated.
 
-    expert(e) returns (W1_e, W3_e, W2_e) as fp64 arrays; shared is None or
-    (Ws1, Ws3, Ws2), the fused always-on MLP of width n_shared * d_ff.
-    Follows the quoted MoE.forward: y starts at zero, every routed expert
-    with at least one token is visited in ascending index and adds
-    gate * expert(x[rows]) to its rows, then the shared MLP output is added
-    to every row. idx_override replaces the selection (gates recomputed from
-    the unbiased scores) to evaluate an alternative valid routing of tied
-    tokens. Returns (y, routing, idx, gates)."""
+    expert(i) returns (W1_i, W3_i, W2_i) as fp64 arrays; shared is None or
+    (Ws1, Ws3, Ws2), the fused shared MLP of width n_shared * d_ff. The sum
+    over i runs in ascending expert index; E_i is evaluated only on the rows
+    where G_i is nonzero (a zero gate adds nothing). idx_override replaces
+    the selection (gates recomputed from the unbiased scores) to evaluate an
+    alternative valid routing of tied tokens. Returns (y, routing, idx,
+    gates)."""
     if routing is None:
         routing = route(x, W_r, b, cfg)
     idx, gates = routing.idx, routing.gates
     if idx_override is not None:
         idx = idx_override.astype(np.int64)
         gates = gates_for(routing.scores, idx, cfg)
-    y = np.zeros_like(x, dtype=np.float64)
-    counts = np.bincount(idx.reshape(-1), minlength=cfg.n_routed)
-    for e in range(cfg.n_routed):
-        if counts[e] == 0:
+    G = gate_matrix(idx, gates, cfg.n_routed)
+    y_routed = np.zeros_like(x, dtype=np.float64)
+    for i in range(cfg.n_routed):
+        rows = np.nonzero(G[:, i])[0]
+        if rows.size == 0:
             continue
-        rows, slot = np.where(idx == e)
-        W1, W3, W2 = expert(e)
-        y[rows] += expert_ffn(x[rows], W1, W3, W2) * gates[rows, slot][:, None]
-    if shared is not None:
-        Ws1, Ws3, Ws2 = shared
-        y += expert_ffn(x, Ws1, Ws3, Ws2)
-    return y, routing, idx, gates
+        y_routed[rows] += G[rows, i][:, None] * expert_ffn(x[rows], *expert(i))
+    y_shared = 0.0 if shared is None else expert_ffn(x, *shared)
+    return y_routed + y_shared, routing, idx, gates
 
 
 # ------------------------------------------------- counts the pages print ----

@@ -88,6 +88,18 @@ def test_score_and_activation_closed_forms():
     np.testing.assert_allclose(P2[:, 0], 1.0 / (1.0 + np.exp(b - a)), rtol=1e-14)
 
 
+def test_score_value_pins():
+    # values, not only symmetries: sigma(ln 3) = 1 / (1 + 1/3) = 3/4, sigma(-ln 3) = 1/4,
+    # silu(ln 3) = (3/4) ln 3 (a wrong slope such as 1/(1+exp(-2z)) gives 9/10 instead);
+    # softmax of (ln 1, ln 2, ln 3) = (1, 2, 3) / 6
+    l3 = math.log(3.0)
+    assert abs(oracle.sigmoid(np.array([l3]))[0] - 0.75) < 1e-15
+    assert abs(oracle.sigmoid(np.array([-l3]))[0] - 0.25) < 1e-15
+    assert abs(oracle.silu(np.array([l3]))[0] - 0.75 * l3) < 1e-15
+    np.testing.assert_allclose(oracle.softmax(np.log(np.array([[1.0, 2.0, 3.0]]))), [[1 / 6, 2 / 6, 3 / 6]],
+                               rtol=1e-15)
+
+
 def test_router_logits_is_x_times_router_rows():
     # z_e is the dot product of the token with centroid e (walkthrough Step 2)
     rng = _rng(2)
@@ -239,6 +251,33 @@ def test_bias_steers_selection_but_not_gates():
     np.testing.assert_allclose(r_f.scores[:, 5], s5, rtol=1e-15)
 
 
+def test_gates_for_hand_example():
+    # scores 0.1 .. 0.4, selection (3, 1): normalised gates 2.5 * (0.4, 0.2) / 0.6 = (5/3, 5/6);
+    # raw gates are route_scale times the selected scores
+    s = np.array([[0.1, 0.2, 0.3, 0.4]])
+    idx = np.array([[3, 1]])
+    cfg_n = RouterCfg(n_routed=4, top_k=2, score="sigmoid", normalize=True, route_scale=2.5)
+    np.testing.assert_allclose(oracle.gates_for(s, idx, cfg_n), [[5 / 3, 5 / 6]], rtol=1e-15)
+    cfg_r = RouterCfg(n_routed=4, top_k=2, score="softmax", route_scale=2.0)
+    np.testing.assert_allclose(oracle.gates_for(s, idx, cfg_r), [[0.8, 0.4]], rtol=1e-15)
+
+
+@pytest.mark.parametrize("score,normalize,scale,G,TG", [("sigmoid", True, 2.5, 8, 4), ("softmax", False, 1.0, 1, 1),
+                                                       ("sigmoid", False, 1.5, 4, 2), ("softmax", True, 1.0, 1, 1)])
+def test_gates_for_reproduces_router_gates(score, normalize, scale, G, TG):
+    # the gates the parity checker recomputes for a given selection equal the
+    # router's own gates when handed the router's own selection, bit for bit
+    rng = _rng(32)
+    N, T, d = 32, 64, 16
+    x = rng.standard_normal((T, d))
+    W = rng.standard_normal((N, d)) / math.sqrt(d)
+    b = rng.uniform(-0.1, 0.1, N)
+    cfg = RouterCfg(n_routed=N, top_k=6, score=score, n_groups=G, topk_groups=TG, normalize=normalize,
+                    route_scale=scale)
+    r = oracle.route(x, W, b, cfg)
+    assert np.array_equal(oracle.gates_for(r.scores, r.idx, cfg), r.gates)
+
+
 # ------------------------------------------------------------ layer level ----
 
 def _layer(rng, T, d, F, N, k, score, ns=0, normalize=False, route_scale=1.0, G=1, TG=1, bias=False):
@@ -276,6 +315,48 @@ def test_identical_experts_normalized_gates_give_route_scale_times_ffn_plus_shar
     # dropping the shared term must show
     y0, *_ = oracle.forward(x, W_r, b, cfg, lambda e: (W1[3], W3[3], W2[3]), None)
     assert np.abs(y - y0).max() > 1e-3
+
+
+def test_idx_override_with_own_selection_is_plain_forward():
+    # re-evaluating a layer with the router's own selection changes nothing (bitwise)
+    rng = _rng(48)
+    T, d, F, N = 24, 12, 10, 16
+    x, W_r, b, (W1, W3, W2), shared, cfg = _layer(rng, T, d, F, N, 4, "sigmoid", ns=1, normalize=True,
+                                                  route_scale=2.5, G=4, TG=2, bias=True)
+    ex = lambda e: (W1[e], W3[e], W2[e])  # noqa: E731
+    y, r, idx, gates = oracle.forward(x, W_r, b, cfg, ex, shared)
+    y2, r2, idx2, gates2 = oracle.forward(x, W_r, b, cfg, ex, shared, idx_override=r.idx)
+    assert np.array_equal(y2, y) and np.array_equal(idx2, idx) and np.array_equal(gates2, gates)
+    # a shuffled slot order of the same selection is the same layer output
+    perm = np.stack([rng.permutation(4) for _ in range(T)])
+    y3, *_ = oracle.forward(x, W_r, b, cfg, ex, shared, idx_override=np.take_along_axis(r.idx, perm, axis=1))
+    np.testing.assert_allclose(y3, y, rtol=1e-13, atol=1e-14)
+
+
+def test_exact_tie_swapped_selection_hand_computed():
+    # d = 2, d_ff = 1, three experts, top-1, sigmoid, raw gates. Experts 1 and 2
+    # have the same router row (ln 3, 0), expert 0 a zero row, so for x = (1, 0)
+    # the scores are (1/2, 3/4, 3/4): an exact tie between 1 and 2, which the
+    # router resolves toward the lower index. Both experts have W1 = (ln 3, 0),
+    # so g = ln 3 and silu(g) = (3/4) ln 3; W3 = (2, 0) / (4, 0) and
+    # W2 = (1, 0)^T / (0, 1)^T give E_1 = (1.5 ln 3, 0) and E_2 = (0, 3 ln 3).
+    # Gate 3/4: y = (9/8 ln 3, 0) with expert 1, (0, 9/4 ln 3) with expert 2.
+    l3 = math.log(3.0)
+    W_r = np.array([[0.0, 0.0], [l3, 0.0], [l3, 0.0]])
+    W1 = np.array([[[l3, 0.0]], [[l3, 0.0]], [[l3, 0.0]]])
+    W3 = np.array([[[1.0, 0.0]], [[2.0, 0.0]], [[4.0, 0.0]]])
+    W2 = np.array([[[1.0], [1.0]], [[1.0], [0.0]], [[0.0], [1.0]]])
+    x = np.array([[1.0, 0.0], [1.0, 0.0]])
+    cfg = RouterCfg(n_routed=3, top_k=1, score="sigmoid")
+    ex = lambda e: (W1[e], W3[e], W2[e])  # noqa: E731
+    y, r, idx, gates = oracle.forward(x, W_r, None, cfg, ex)
+    assert r.sel_tie.all() and idx.tolist() == [[1], [1]]
+    np.testing.assert_allclose(gates, [[0.75], [0.75]], rtol=1e-15)
+    np.testing.assert_allclose(y, [[9 / 8 * l3, 0.0], [9 / 8 * l3, 0.0]], rtol=1e-14, atol=1e-15)
+    # the other valid selection for token 1 only
+    y2, _, idx2, gates2 = oracle.forward(x, W_r, None, cfg, ex, routing=r, idx_override=np.array([[1], [2]]))
+    np.testing.assert_allclose(gates2, [[0.75], [0.75]], rtol=1e-15)
+    np.testing.assert_allclose(y2, [[9 / 8 * l3, 0.0], [0.0, 9 / 4 * l3]], rtol=1e-14, atol=1e-15)
 
 
 def test_segmentation_identity_single_expert():
