@@ -4,9 +4,14 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours
 
 One step = one moe_forward over one batch of T synthetic tokens (router,
 dispatch, row gather, SwiGLU GEMM, gate GEMM, combine), weights resident in
-HBM. With N > 1 (torchrun, one process per GPU) every rank runs its own batch
-on a full replica of the weights: data-parallel, no collective on the data
-path (weak scaling); timing is the max over ranks. Rank 0 prints one JSON line.
+HBM. The timed loop calls moe_forward exactly as a user does (no per-stage
+events, so the two GEMMs overlap through programmatic dependent launch); a
+second, shorter pass with stage events gives the per-kernel times. With
+--gpus N > 1 the script starts N local ranks itself (torch.distributed.run)
+unless it already runs under torchrun; every rank runs its own batch on a full
+replica of the weights: data-parallel, no collective on the data path (weak
+scaling); timing is the max over ranks. Rank 0 prints one JSON line, with the
+V3 decode layer timed the same way in its "decode" object.
 
 The reference arm (--impl reference) times the fp64 CPU oracle on a bounded
 sample of the same workload on the host cores.
@@ -18,6 +23,7 @@ import hashlib
 import json
 import math
 import os
+import socket
 import subprocess
 import sys
 import threading
@@ -82,57 +88,64 @@ def ncu_traffic(config: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """SM clock and clock-event reasons of one GPU, polled through NVML every
+    few milliseconds while the timed region runs (nvidia-smi's 200 ms period
+    gives a single sample over a 0.1 s region)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_id):
-        self.gpu = gpu_id
-        self.proc = None
-        self.lines = []
+    def __init__(self, uuid, period_s=0.003):
+        self.uuid = uuid
+        self.period = period_s
+        self.samples = []
+        self.handle = None
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.t = None
 
     def __enter__(self):
         try:
-            sel = [f"--id={self.gpu}"] if self.gpu else []
-            self.proc = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = (pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid
+                           else pynvml.nvmlDeviceGetHandleByIndex(0))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            self.t = threading.Thread(target=self._poll, daemon=True)
             self.t.start()
-        except OSError:
-            self.proc = None
+        except Exception:  # no NVML: the line reports the clocks as unsampled
+            self.handle = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _poll(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                why = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((float(mhz), int(why)))
+            except Exception:
+                break
+            self._stop.wait(self.period)
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self.t is not None:
+            self.t.join(timeout=5)
 
     def summary(self):
-        rows = []
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v.lower() == "active"})
-        return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": rows[0][1],
-                "reasons": reasons, "samples": len(rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0}
+        mhz = [m for m, _ in self.samples]
+        seen = {}
+        for _, why in self.samples:
+            for bit, name in self.REASONS.items():
+                if why & bit:
+                    seen[name] = seen.get(name, 0) + 1
+        return {"sm_mhz": float(np.median(mhz)), "sm_min_mhz": float(min(mhz)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(seen), "reason_samples": seen, "samples": len(self.samples),
+                "source": "NVML, every ~3 ms over the timed region"}
 
 
 def rank_env():
@@ -158,26 +171,116 @@ def max_over_ranks(values, device=None):
 
 
 def algorithmic(s: mi.LayerShape, counts: np.ndarray):
-    """FLOPs and HBM bytes the layer must move (touched expert weights, router
-    weights, x read, y written), and the SwiGLU GEMM's own bytes."""
+    """What the layer must do, independent of how: FLOPs of the expert
+    matmuls, HBM bytes of the layer (touched expert weights, router weights,
+    x read, y written), and the SwiGLU GEMM's bytes counted two ways --
+    touched W1/W3 weights plus x read once (the algorithmic count), and that
+    plus the implementation's own token-row reads and SwiGLU-row writes."""
     U = int((counts > 0).sum())
     e = 2 if s.dtype == "bf16" else 4
     flops = s.T * (s.top_k + s.n_shared) * 6 * s.d * s.d_ff
     layer_bytes = (U + s.n_shared) * 3 * s.d * s.d_ff * e + s.n_routed * s.d * e + 2 * s.T * s.d * e
     R = s.T * s.top_k
-    swiglu_bytes = ((U + s.n_shared) * 2 * s.d * s.d_ff * e          # W1, W3 of touched experts
-                    + (R + (s.T if s.n_shared else 0)) * s.d * e       # token rows read
-                    + (R * s.d_ff + s.T * s.n_shared * s.d_ff) * e)    # SwiGLU rows written
-    return U, flops, layer_bytes, swiglu_bytes
+    w13 = (U + s.n_shared) * 2 * s.d * s.d_ff * e
+    swiglu_alg = w13 + s.T * s.d * e
+    swiglu_impl = (w13 + (R + (s.T if s.n_shared else 0)) * s.d * e
+                   + (R * s.d_ff + s.T * s.n_shared * s.d_ff) * e)
+    return {"U": U, "flops": flops, "layer_bytes": layer_bytes, "swiglu_alg": swiglu_alg,
+            "swiglu_impl": swiglu_impl}
+
+
+class Layer:
+    """One layer configuration on the device: weights, a token batch, a
+    workspace, and the moe_forward / moe_forward_host calls a user makes."""
+
+    def __init__(self, s: mi.LayerShape, rank: int):
+        import torch
+        import mixture_experts_layer_group_b200 as moe
+        from moe_inputs import device as mdev
+        self.moe = moe
+        self.s = s
+        self.w = mdev.device_all(s)  # the same replica on every rank
+        self.x = mdev.device_tensor(token_shape_for_rank(s, rank), "x")
+        self.cfg = moe.make_cfg(s.d, s.d_ff, s.n_routed, s.n_shared, s.top_k, s.n_groups, s.topk_groups, s.score,
+                                s.normalize, s.route_scale, s.group_score, s.dtype)
+        self.ws = torch.empty(moe.workspace_size_host(self.cfg, s.T), dtype=torch.uint8, device="cuda")
+        self.y = torch.empty_like(self.x)
+        self.stream = torch.cuda.current_stream()
+        w = self.w
+        self.wargs = (w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"])
+
+    def step(self):
+        self.moe.forward(self.cfg, self.s.T, self.x, *self.wargs, self.y, self.ws, stream=self.stream)
+
+    def routing_counts(self):
+        import torch
+        s = self.s
+        idx = torch.empty((s.T, s.top_k), dtype=torch.int32, device="cuda")
+        gates = torch.empty((s.T, s.top_k), dtype=torch.float32, device="cuda")
+        self.moe.forward(self.cfg, s.T, self.x, *self.wargs, self.y, self.ws, idx, gates, stream=self.stream)
+        torch.cuda.synchronize()
+        status = self.moe.device_status(self.cfg, s.T, self.ws)
+        return np.bincount(idx.cpu().numpy().reshape(-1), minlength=s.n_routed), status
+
+    def timed(self, steps, clk=None):
+        """ms per step of `steps` back-to-back moe_forward calls, CUDA events on the launching stream."""
+        import torch
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        t0.record(self.stream)
+        for _ in range(steps):
+            self.step()
+        t1.record(self.stream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / steps
+
+    def stage_pass(self, steps):
+        """Per-stage ms (mean over `steps` calls) from the library's stage
+        events; with events between the GEMMs the down GEMM starts after the
+        SwiGLU GEMM instead of overlapping its drain."""
+        import torch
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
+        for row in ev:
+            for e in row:
+                e.record(self.stream)
+        torch.cuda.synchronize()
+        for k in range(steps):
+            self.moe.set_stage_events(ev[k])
+            self.step()
+        self.moe.set_stage_events(None)
+        torch.cuda.synchronize()
+        return {name: float(np.mean([ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)]))
+                for i, name in enumerate(self.moe.STAGES)}
+
+    def e2e(self, steps, warmup):
+        """ms per step through moe_forward_host: x copied in from pinned host
+        memory and y copied back to it on every step."""
+        import torch
+        xh = self.x.cpu().pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+        for _ in range(warmup):
+            self.moe.forward_host(self.cfg, self.s.T, xh, *self.wargs, yh, self.ws, stream=self.stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for _ in range(steps):
+            self.moe.forward_host(self.cfg, self.s.T, xh, *self.wargs, yh, self.ws, stream=self.stream)
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        self.moe.workspace_release(self.ws)
+        return e0.elapsed_time(e1) / steps, xh.numel() * xh.element_size(), yh.numel() * yh.element_size()
+
+    def free(self):
+        import torch
+        self.w = self.x = self.ws = self.y = self.wargs = None
+        torch.cuda.empty_cache()
 
 
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
-    import mixture_experts_layer_group_b200 as moe
     from mixture_experts_layer_group_b200 import build as lib_build
     from moe_inputs import build as gen_build
-    from moe_inputs import device as mdev
 
     if rank == 0 or world == 1:
         lib_build.build()
@@ -186,92 +289,66 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.set_device(local_rank)
     s = mi.SHAPES[args.config]
-    # weights are the same replica everywhere; each rank draws its own token batch
-    sx = token_shape_for_rank(s, rank)
-    w = mdev.device_all(s)
-    x = mdev.device_tensor(sx, "x")
-    cfg = moe.make_cfg(s.d, s.d_ff, s.n_routed, s.n_shared, s.top_k, s.n_groups, s.topk_groups, s.score,
-                       s.normalize, s.route_scale, s.group_score, s.dtype)
-    ws = torch.empty(moe.workspace_size_host(cfg, s.T), dtype=torch.uint8, device="cuda")
-    y = torch.empty_like(x)
-    idx = torch.empty((s.T, s.top_k), dtype=torch.int32, device="cuda")
-    gates = torch.empty((s.T, s.top_k), dtype=torch.float32, device="cuda")
-    stream = torch.cuda.current_stream()
-    wargs = (w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"])
-
-    def step():
-        moe.forward(cfg, s.T, x, *wargs, y, ws, stream=stream)
-
+    L = Layer(s, rank)
     for _ in range(args.warmup):
-        step()
-    moe.forward(cfg, s.T, x, *wargs, y, ws, idx, gates, stream=stream)
-    torch.cuda.synchronize()
-    status = moe.device_status(cfg, s.T, ws)
-    counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=s.n_routed)
+        L.step()
+    counts, status = L.routing_counts()
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(local_rank).uuid)
+    except Exception:
+        uuid = None
 
-    # --- device-timed region: K steps, stage events on the launching stream
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
-    for row in ev:
-        for e in row:
-            e.record(stream)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # --- device-timed region: K product-path steps (no stage events)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local_rank).uuid)
-    except Exception:
-        gpu_id = None
-    with ClockSampler(gpu_id) as clk:
+    with ClockSampler(uuid) as clk:
         wall0 = time.perf_counter()
-        t0.record(stream)
-        for k in range(args.steps):
-            moe.set_stage_events(ev[k])
-            step()
-        t1.record(stream)
-        moe.set_stage_events(None)
-        torch.cuda.synchronize()
+        ms = L.timed(args.steps)
         wall = time.perf_counter() - wall0
     if world > 1:
         dist.barrier()
-    ms = t0.elapsed_time(t1) / args.steps
-    stage_ms = {name: float(np.mean([ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)]))
-                for i, name in enumerate(moe.STAGES)}
+    # --- per-kernel times (separate pass with stage events)
+    stage_ms = L.stage_pass(min(args.steps, 20))
+    # --- end to end through the host-buffer entry point
+    e2e_ms, h2d, d2h = L.e2e(args.steps, max(1, args.warmup // 2))
+    L.free()
 
-    # --- end to end: host tokens in, host output back, every step
-    xh = x.cpu().pin_memory()
-    yh = torch.empty_like(xh).pin_memory()
-    for _ in range(max(1, args.warmup // 2)):
-        moe.forward_host(cfg, s.T, xh, *wargs, yh, ws, stream=stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        moe.forward_host(cfg, s.T, xh, *wargs, yh, ws, stream=stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
+    # --- the V3 decode layer, timed the same way
+    dec = None
+    if not args.no_decode and args.config != "v3_decode_bf16":
+        ds = mi.SHAPES["v3_decode_bf16"]
+        D = Layer(ds, rank)
+        for _ in range(args.warmup):
+            D.step()
+        dcounts, dstatus = D.routing_counts()
+        if world > 1:
+            dist.barrier()
+        with ClockSampler(uuid) as dclk:
+            dms = D.timed(args.steps)
+        dstage = D.stage_pass(min(args.steps, 20))
+        D.free()
+        dec = (ds, dms, dcounts, dstatus, dstage, dclk.summary())
 
-    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device="cuda")
+    vals = [ms, e2e_ms] + ([dec[1]] if dec else [])
+    vals = max_over_ranks(vals, device="cuda")
+    ms, e2e_ms = vals[0], vals[1]
     if rank != 0:
         return None
 
     peaks, peak_src = load_peaks()
-    U, flops, layer_bytes, swiglu_bytes = algorithmic(s, counts)
+    A = algorithmic(s, counts)
     t_sec = ms / 1e3
-    tok_s = world * s.T / t_sec
-    tflops = flops / t_sec / 1e12
-    gbs = layer_bytes / t_sec / 1e9
-    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
-    t_hbm = layer_bytes / (peaks["hbm_gbs"] * 1e9)
+    tflops = A["flops"] / t_sec / 1e12
+    gbs = A["layer_bytes"] / t_sec / 1e9
+    t_tc = A["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_hbm = A["layer_bytes"] / (peaks["hbm_gbs"] * 1e9)
     sw_ms = stage_ms["gemm_swiglu"]
-    achieved = swiglu_bytes / (sw_ms / 1e3) / 1e9
-    clocks = clk.summary()
+    achieved = A["swiglu_alg"] / (sw_ms / 1e3) / 1e9
+    achieved_impl = A["swiglu_impl"] / (sw_ms / 1e3) / 1e9
     out = {
         "metric": METRIC,
-        "value": round(tok_s, 1),
+        "value": round(world * s.T / t_sec, 1),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -286,26 +363,45 @@ def run_ours(args, rank, world, local_rank):
                    "n_shared": s.n_shared, "d_ff": s.d_ff, "top_k": s.top_k, "global_batch": world * s.T,
                    "parallelism": f"dp{world} (independent replicas, no collective)",
                    "l2": "inputs larger than L2: every step streams "
-                         f"{(U + s.n_shared) * 3 * s.d * s.d_ff * 2 / 1e9:.1f} GB of expert weights"},
+                         f"{(A['U'] + s.n_shared) * 3 * s.d * s.d_ff * 2 / 1e9:.1f} GB of expert weights"},
         "e2e": {"value": round(world * s.T / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": s.T * s.d * (2 if s.dtype == "bf16" else 4),
-                "d2h_bytes_per_step": s.T * s.d * (2 if s.dtype == "bf16" else 4)},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+                "api": "moe_forward_host (pinned host x in, y out, every step)"},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "roofline": {"bound": "hbm", "kernel": "expert_gemm_tc_kernel<SwiGLU>",
                      "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": ncu_traffic(args.config),
                      "peak_source": f"hbm_gbs, {peak_src}", "launch_ms": round(sw_ms, 4),
-                     "algorithmic_bytes": swiglu_bytes},
-        "layer": {"tflops": round(tflops, 1), "tc_frac_of_sustained": round(tflops * 1e12 / (peaks["bf16_tflops_sustained"] * 1e12), 4),
+                     "algorithmic_bytes": A["swiglu_alg"],
+                     "counting": "touched W1/W3 weights + x read once; launch_ms from the stage pass",
+                     "impl_bytes": A["swiglu_impl"], "impl_frac": round(achieved_impl / peaks["hbm_gbs"], 4)},
+        "layer": {"tflops": round(tflops, 1),
+                  "tc_frac_of_sustained": round(tflops * 1e12 / (peaks["bf16_tflops_sustained"] * 1e12), 4),
                   "hbm_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
                   "binding_roofline_ms": round(max(t_tc, t_hbm) * 1e3, 4),
                   "binding_frac": round(max(t_tc, t_hbm) / t_sec, 4),
                   "bound": "hbm" if t_hbm > t_tc else "tensor",
-                  "touched_routed_experts": U, "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()}},
-        "clocks": clocks,
+                  "touched_routed_experts": A["U"], "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+                  "stage_pass": "separate pass with stage events (down GEMM not overlapped)"},
+        "clocks": clk.summary(),
         "device_status": status,
         "wall_s_timed": round(wall, 3),
     }
+    if dec:
+        ds, dms, dcounts, dstatus, dstage, dclocks = dec
+        dms = vals[2]
+        DA = algorithmic(ds, dcounts)
+        dt = dms / 1e3
+        d_t_hbm = DA["layer_bytes"] / (peaks["hbm_gbs"] * 1e9)
+        d_t_tc = DA["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+        out["decode"] = {"workload": describe(ds), "ms_per_step": round(dms, 4),
+                         "tokens_per_s": round(world * ds.T / dt, 1), "touched_routed_experts": DA["U"],
+                         "hbm_gbs": round(DA["layer_bytes"] / dt / 1e9, 1),
+                         "hbm_frac": round(DA["layer_bytes"] / dt / 1e9 / peaks["hbm_gbs"], 4),
+                         "binding_frac": round(max(d_t_hbm, d_t_tc) / dt, 4),
+                         "bound": "hbm" if d_t_hbm > d_t_tc else "tensor",
+                         "bytes": DA["layer_bytes"], "stage_ms": {k: round(v, 4) for k, v in dstage.items()},
+                         "clocks": dclocks, "device_status": dstatus}
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(s, args.cpu_tokens)
     return out
@@ -459,6 +555,37 @@ def run_router_only(args):
             "router_tflops": round(flops / (ms * 1e-3) / 1e12, 2), "config": {"workload": s.name, "T": s.T}}
 
 
+def free_port() -> int:
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_ranks(n: int, argv) -> int:
+    """Re-run this script as n local ranks, one process per GPU, through
+    torch.distributed.run on 127.0.0.1; returns the launcher's exit code."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def check_launch(world: int, rank: int) -> int:
+    """The rank plumbing alone: every rank joins a gloo group, rank 0 prints
+    the ranks it saw."""
+    import datetime
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        seen = [None] * world
+        dist.all_gather_object(seen, {"rank": rank, "pid": os.getpid()})
+        dist.destroy_process_group()
+    else:
+        seen = [{"rank": 0, "pid": os.getpid()}]
+    if rank == 0:
+        print(json.dumps({"n_gpus": world, "ranks": seen}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -468,12 +595,19 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the V3 decode sub-measurement")
+    ap.add_argument("--check-launch", action="store_true",
+                    help="start the ranks, join a gloo process group, report them and exit (no GPU work)")
     ap.add_argument("--stage", default="layer", choices=["layer", "router", "bias"],
                     help="router: time moe_route alone; bias: time moe_bias_update (profiling aids; 1 GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv))
     world, rank, local_rank = rank_env()
+    if args.check_launch:
+        return check_launch(world, rank)
     if args.stage in ("router", "bias"):
         print(json.dumps(run_router_only(args)), flush=True)
         return 0

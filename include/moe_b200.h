@@ -73,7 +73,11 @@ enum {
   MOE_DEV_WAIT_TIMEOUT = 1u << 0,   /* a bounded pipeline wait gave up */
   MOE_DEV_BAD_EXPERT = 1u << 1,     /* an expert index outside [0, n_routed) */
   MOE_DEV_DUP_EXPERT = 1u << 2,     /* a token lists the same expert twice */
-  MOE_DEV_TMEM_ALLOC = 1u << 3      /* tensor-memory allocation returned no columns */
+  MOE_DEV_TMEM_ALLOC = 1u << 3,     /* tensor-memory allocation returned no columns */
+  MOE_DEV_NONFINITE = 1u << 4       /* a token's router logits or keys were NaN or infinite
+                                       (non-finite x, W_r or b); it still gets top_k distinct
+                                       experts in [0, n_routed), chosen arbitrarily, and the
+                                       other tokens are unaffected */
 };
 
 /*
@@ -173,17 +177,31 @@ MOE_API moe_status moe_forward(const moe_cfg* cfg, int64_t T, const void* x, con
  * caller synchronises the stream before reading y_host. Weights stay in
  * device memory. Needs moe_workspace_size_host() bytes of workspace.
  * The host-to-device copy runs on a copy stream the library keeps for the
- * workspace (with two events; created on first use, kept until the process
- * exits) and waits only until the previous call on the same workspace has
- * finished reading its staged x, so back-to-back calls overlap one call's
- * input copy with the previous call's down projection and output copy. The
- * output copy stays on `stream`.
+ * workspace (with four events, no device memory; created on the first host
+ * call on that workspace, freed by moe_workspace_release or at process exit).
+ * x is staged in two slots used by alternate calls, so back-to-back calls
+ * with the same T and cfg overlap one call's input copy with the whole of
+ * the previous call. A call with another T or cfg, or one that follows a
+ * moe_route / moe_dispatch / moe_forward call on the same workspace, waits
+ * for the previous call to finish before copying (its staging area may then
+ * overlap buffers that call still uses). The output copy stays on `stream`.
+ * All calls on one workspace must be ordered: issue them on one stream, or
+ * order the streams yourself.
  */
 MOE_API moe_status moe_workspace_size_host(const moe_cfg* cfg, int64_t T, size_t* bytes);
 MOE_API moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
                             const float* b, const void* W1, const void* W3, const void* W2,
                             const void* Ws1, const void* Ws3, const void* Ws2, void* y_host,
                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Frees the copy stream and events that moe_forward_host keeps for the
+ * workspace at `ws` (nothing happens if it has none). Call it before freeing
+ * or reusing that memory for another purpose; work still queued on the
+ * stream completes first. The workspace memory itself belongs to the caller.
+ * Errors: MOE_ERR_CUDA if the workspace's device cannot be made current.
+ */
+MOE_API moe_status moe_workspace_release(const void* ws);
 
 /*
  * Reads (and optionally clears) the device-status word of a workspace used
@@ -211,16 +229,21 @@ MOE_API moe_status moe_set_stage_events(void* const* events, int32_t n);
  * memory and passes it no workspace, or a serving loop with a fixed memory
  * budget that must not call cudaMalloc (which can synchronise the device)
  * once it runs.
- *   Same arguments, outputs and results as moe_route, without ws/ws_bytes.
- *   Scratch: the fp32 logits (T * n_routed * 4 bytes) go to a fixed 8 MiB
- *     array inside the library, reserved on every GPU that loads the
- *     library until the process exits. T * n_routed * 4 > 8 MiB (for
- *     example T > 8192 at n_routed = 256) returns MOE_ERR_UNSUPPORTED; use
- *     moe_route with a workspace for those sizes.
+ *   Same arguments and outputs as moe_route, without ws/ws_bytes, and the
+ *     same results bit for bit: the logits are reduced in the same K ranges
+ *     as moe_route's (when moe_route's partial logits for all T tokens do not
+ *     fit the array, the router runs over slices of the tokens in turn).
+ *   Scratch: the fp32 logits go to a fixed 8 MiB array inside the library,
+ *     reserved on every GPU that loads the library until the process exits.
+ *     T * n_routed * 4 > 8 MiB (for example T > 8192 at n_routed = 256)
+ *     returns MOE_ERR_UNSUPPORTED before any device work; use moe_route
+ *     with a workspace for those sizes.
  *   Set-up: the first call on a device (with that device current) looks up
  *     the array's device address and caches it; make that first call before
  *     any stream capture. It never calls cudaMalloc, cudaFree or any other
- *     allocating routine.
+ *     allocating routine. The cached address belongs to the device's
+ *     current primary context: after cudaDeviceReset() on a device, this
+ *     call must not be used on that device again in the same process.
  *   Sharing: every call on a device uses the same array and leaves the last
  *     call's logits in it (each call overwrites every value it reads, so
  *     nothing needs clearing). Calls whose work overlaps on the GPU -- on
@@ -259,6 +282,8 @@ MOE_API moe_status moe_bias_update(const moe_cfg* cfg, int64_t T, const int32_t*
  * limit (1 s) the kernel records MOE_DEV_WAIT_TIMEOUT and returns; the call
  * synchronises `stream` and writes the recorded bits to *bits (expected:
  * MOE_DEV_WAIT_TIMEOUT). The CUDA context stays usable. Takes about 1 s.
+ * Calls from different host threads of one process are serialised inside
+ * the library (they share one status word per device).
  * Errors: MOE_ERR_INVALID_ARG for a null bits; MOE_ERR_CUDA for a failed
  * launch or copy.
  */

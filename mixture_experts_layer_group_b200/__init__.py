@@ -18,11 +18,11 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_F32, MOE_BF16 = 0, 1
 MOE_SOFTMAX, MOE_SIGMOID = 0, 1
 MOE_GROUP_TOP2_SUM, MOE_GROUP_MAX = 0, 1
-MOE_DEV_WAIT_TIMEOUT, MOE_DEV_BAD_EXPERT, MOE_DEV_DUP_EXPERT, MOE_DEV_TMEM_ALLOC = 1, 2, 4, 8
+MOE_DEV_WAIT_TIMEOUT, MOE_DEV_BAD_EXPERT, MOE_DEV_DUP_EXPERT, MOE_DEV_TMEM_ALLOC, MOE_DEV_NONFINITE = 1, 2, 4, 8, 16
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE"}
 EXPORTS = ["moe_workspace_size", "moe_workspace_size_host", "moe_route", "moe_dispatch", "moe_forward",
-           "moe_forward_host", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update", "moe_selftest_wait_timeout",
+           "moe_forward_host", "moe_workspace_release", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update", "moe_selftest_wait_timeout",
            "moe_status_string", "moe_last_cuda_error"]
 STAGES = ["router", "dispatch", "gather", "gemm_swiglu", "gemm_gate", "combine"]
 
@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
         L.moe_dispatch.argtypes = [CFG, I64, P, P, P, P, P, SZ, P]
         L.moe_forward.argtypes = [CFG, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.moe_forward_host.argtypes = [CFG, I64, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_workspace_release.argtypes = [P]
         L.moe_device_status.argtypes = [CFG, I64, P, SZ, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32), P]
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
         L.moe_route_noalloc.argtypes = [CFG, I64, P, P, P, P, P, P]
@@ -82,12 +83,25 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
+_SCORES = {"softmax": MOE_SOFTMAX, "sigmoid": MOE_SIGMOID}
+_GROUP_SCORES = {"top2_sum": MOE_GROUP_TOP2_SUM, "max": MOE_GROUP_MAX}
+_DTYPES = {"bf16": MOE_BF16, "f32": MOE_F32}
+
+
+def _lookup(table: dict, what: str, value: str) -> int:
+    try:
+        return table[value]
+    except KeyError:
+        raise ValueError(f"unknown {what} {value!r}; expected one of {sorted(table)}") from None
+
+
 def make_cfg(d, d_ff, n_routed, n_shared, top_k, n_groups=1, topk_groups=1, score="softmax",
              normalize=False, route_scale=1.0, group_score="top2_sum", dtype="bf16") -> MoeCfg:
-    return MoeCfg(d, d_ff, n_routed, n_shared, top_k, n_groups, topk_groups,
-                  MOE_SIGMOID if score == "sigmoid" else MOE_SOFTMAX, int(bool(normalize)),
-                  float(route_scale), MOE_GROUP_MAX if group_score == "max" else MOE_GROUP_TOP2_SUM,
-                  MOE_BF16 if dtype == "bf16" else MOE_F32)
+    """moe_cfg from Python values; an unknown score, group_score or dtype
+    string raises ValueError instead of falling back to a default."""
+    return MoeCfg(d, d_ff, n_routed, n_shared, top_k, n_groups, topk_groups, _lookup(_SCORES, "score", score),
+                  int(bool(normalize)), float(route_scale), _lookup(_GROUP_SCORES, "group_score", group_score),
+                  _lookup(_DTYPES, "dtype", dtype))
 
 
 def _ptr(t):
@@ -176,6 +190,11 @@ def forward_host(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, 
                                                       _ptr(W1), _ptr(W3), _ptr(W2), _ptr(Ws1), _ptr(Ws3),
                                                       _ptr(Ws2), _ptr(y_host), _ptr(ws), ws_bytes,
                                                       _stream(stream)))
+
+
+def workspace_release(ws) -> None:
+    """Free the copy stream and events moe_forward_host keeps for this workspace."""
+    _check("moe_workspace_release", lib().moe_workspace_release(_ptr(ws)))
 
 
 def device_status(cfg, T, ws, clear=True, ws_bytes=None, stream=None) -> int:

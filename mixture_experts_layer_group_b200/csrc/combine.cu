@@ -1,9 +1,11 @@
 // Combine: y[t] = sum of the gated expert rows of token t, in ascending
 // expert index, plus the shared-MLP row, accumulated in fp32 and rounded
-// once (the quoted MoE.forward's fp32 accumulator and its expert loop in
-// ascending index, then "y += shared_experts(x)"; "DeepSeek-V3.2-Exp ·
-// Mixture of experts", Delta_ffn = y_routed + y_shared). A fixed order and
-// no atomics make the result bitwise reproducible.
+// once. This is the last step of the "All 19 steps" list on the
+// "DeepSeek-V3.2-Exp · Mixture of experts" page (Delta_ffn = y_routed +
+// y_shared, with y_routed the gate-weighted sum over the selected experts);
+// the fp32 accumulator and the ascending expert order follow the same page's
+// quoted forward excerpt. A fixed order and no atomics make the result
+// bitwise reproducible.
 #include "common.cuh"
 #include "internal.h"
 

@@ -214,20 +214,26 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a, int32_t* chunk_b
   }
 }
 
-template <typename TV>
+// x_perm[slot_pos[t, s]] = x[t] for every placed pair: one warp per token
+// reads its row once and writes it to each of its k permuted rows, so x is
+// read from HBM once (a pair left at -1 by an invalid index is skipped).
+template <typename TV, int KMAX>
 __global__ void __launch_bounds__(256) gather_kernel(const TV* __restrict__ x,
-                                                     const int32_t* __restrict__ perm,
-                                                     const int32_t* __restrict__ n_rows, int64_t R,
+                                                     const int32_t* __restrict__ slot_pos, int64_t T,
                                                      int k, int vecs, TV* __restrict__ x_perm) {
   const int lane = threadIdx.x & 31;
-  const int64_t rows = *n_rows;  // pairs actually placed (== R unless the indices were invalid)
-  if (rows < R) R = rows < 0 ? 0 : rows;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += warps) {
-    const int64_t t = perm[r] / k;
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+    int32_t dst[KMAX];
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) dst[s] = s < k ? __ldg(slot_pos + t * k + s) : -1;
     const TV* src = x + t * vecs;
-    TV* dst = x_perm + r * vecs;
-    for (int v = lane; v < vecs; v += 32) dst[v] = src[v];
+    for (int v = lane; v < vecs; v += 32) {
+      const TV val = __ldg(src + v);
+#pragma unroll
+      for (int s = 0; s < KMAX; ++s)
+        if (dst[s] >= 0) x_perm[(int64_t)dst[s] * vecs + v] = val;
+    }
   }
 }
 
@@ -254,15 +260,18 @@ cudaError_t launch_dispatch(const Problem& p, const DispatchBuffers& db, int bm,
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm,
-                          const int32_t* n_rows, void* x_perm, cudaStream_t s) {
+cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* slot_pos, void* x_perm,
+                          cudaStream_t s) {
   if (p.R == 0) return cudaSuccess;
   const int vecs = (int)((int64_t)p.d * p.elem / 16);
-  int64_t want = (p.R + 7) / 8;
-  int64_t cap = (int64_t)device_sm_count() * 16;
-  unsigned blocks = (unsigned)(want < cap ? want : cap);
-  gather_kernel<uint4><<<blocks, 256, 0, s>>>((const uint4*)x, perm, n_rows, p.R, p.k, vecs,
-                                              (uint4*)x_perm);
+  const int64_t want = (p.T + 7) / 8;
+  const int64_t cap = (int64_t)device_sm_count() * 16;
+  const unsigned blocks = (unsigned)(want < cap ? want : cap);
+  if (p.k <= 8)
+    gather_kernel<uint4, 8><<<blocks, 256, 0, s>>>((const uint4*)x, slot_pos, p.T, p.k, vecs, (uint4*)x_perm);
+  else
+    gather_kernel<uint4, kMaxTopK><<<blocks, 256, 0, s>>>((const uint4*)x, slot_pos, p.T, p.k, vecs,
+                                                          (uint4*)x_perm);
   return cudaGetLastError();
 }
 

@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kThreads) expert_gemm_simt_kernel(SimtParams p
 }  // namespace
 
 cudaError_t launch_expert_gemms_simt(const Problem& p, const GemmArgs& a, cudaStream_t s,
-                                   cudaEvent_t between, cudaEvent_t between2) {
+                                   cudaEvent_t between) {
   const int sms = device_sm_count();
   const int grid = sms * 4;
   SimtParams g1{(const float*)a.x_perm, (const float*)a.x, (const float*)a.W1, (const float*)a.W3,
@@ -134,7 +134,6 @@ cudaError_t launch_expert_gemms_simt(const Problem& p, const GemmArgs& a, cudaSt
   expert_gemm_simt_kernel<true><<<grid, kThreads, 0, s>>>(g1);
   cudaError_t err = cudaGetLastError();
   if (err == cudaSuccess && between) err = cudaEventRecord(between, s);
-  if (err == cudaSuccess && between2) err = cudaEventRecord(between2, s);
   if (err != cudaSuccess) return err;
   SimtParams g2{(const float*)a.h_perm, (const float*)a.h_sh, (const float*)a.W2, nullptr,
                 (const float*)a.Ws2, nullptr, a.unit_base2, a.grp_row0, a.grp_rows, p.N, p.F, p.nsF,

@@ -90,24 +90,6 @@ static_assert(kMaxTok <= kBufCols && kMaxTok % (2 * kTokBox) == 0, "token chunk"
 
 enum Mode : int { kSwiGLU = 0, kGateDown = 1 };
 
-// Optional per-unit timestamps (%globaltimer) of the three roles, compiled in
-// only with -DMOE_UNIT_TRACE for pipeline studies; a no-op otherwise.
-#ifdef MOE_UNIT_TRACE
-constexpr int kTraceCtas = 160, kTraceUnits = 160;
-__device__ unsigned long long g_unit_trace[2][kTraceCtas][kTraceUnits][16];
-#define MOE_TRACE_VAL(mode, unit_i, slot, value)                                        \
-  do {                                                                                 \
-    if (blockIdx.x < kTraceCtas && (unit_i) < kTraceUnits)                             \
-      g_unit_trace[mode][blockIdx.x][unit_i][slot] = (value);                          \
-  } while (0)
-#else
-#define MOE_TRACE_VAL(mode, unit_i, slot, value) \
-  do {                                           \
-    (void)(unit_i);                              \
-  } while (0)
-#endif
-#define MOE_TRACE(mode, unit_i, slot) MOE_TRACE_VAL(mode, unit_i, slot, global_timer_ns())
-
 struct TcParams {
   CUtensorMap a0_routed;  // W1 [N*F, d]      | W2 [N*d, F]
   CUtensorMap a1_routed;  // W3 [N*F, d]      | unused
@@ -370,9 +352,6 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         const CUtensorMap* ta1 = MODE == kSwiGLU ? (shared ? &p.a1_shared : &p.a1_routed) : ta0;
         const CUtensorMap* tb = shared ? &p.b_shared[tmap] : &p.b_routed[tmap];
         const uint64_t pol = un.nchunks == 1 ? pol_once : pol_shared;
-        MOE_TRACE(MODE, i, 0);
-        MOE_TRACE_VAL(MODE, i, 7, (unsigned long long)un.ntok | ((unsigned long long)un.tok0 << 16) |
-                                      ((unsigned long long)un.g << 32) | ((unsigned long long)un.f << 48));
         for (int kc = 0; kc < nk; ++kc, ++fills) {
           const uint32_t s = fills % kSlots;
           uint32_t pos = 0;
@@ -391,7 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           tma_load_2d_pair(a_dst + kHalfBytes, ta1, full_bar, kc * kBK, rowA + half_rows, pol);
           tma_load_2d_pair(b_dst, tb, full_bar, kc * kBK, rowB, pol_shared);
         }
-        MOE_TRACE(MODE, i, 1);
         if (!ok) break;
       }
       if (!ok) {
@@ -423,14 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         uint32_t mask, base, stride;
         plan.place(un.ntok, mask, base, stride);
         plan.advance(un.ntok);
-        MOE_TRACE(MODE, i, 2);
         for (int b = 0; b < 2 && ok; ++b)
           if ((mask >> b) & 1u) {
             ok = mbar_wait_cluster_bounded(&sh.acc_empty[b], (uses[b] & 1u) ^ 1u, abort_flag);
             ++uses[b];
           }
         if (!ok) break;
-        MOE_TRACE(MODE, i, 3);
         tc_fence_after();
         const uint32_t d0 = tmem_base + base, d1 = tmem_base + base + stride;
         for (int kc = 0; kc < nk; ++kc) {
@@ -459,7 +435,6 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
               umma_commit_pair(peer(&sh.acc_full[b]));
             }
         }
-        MOE_TRACE(MODE, i, 4);
       }
       if (!ok) {
         *abort_flag = 1;
@@ -528,7 +503,6 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
       plan.advance(un.ntok);
       uses[0] += mask & 1u;
       uses[1] += (mask >> 1) & 1u;
-      if (leader) MOE_TRACE(MODE, i, 5);
       tc_fence_after();
       const bool shared = un.g == p.N;
       const int64_t row_base = load_volatile(&sh.epi_info[i & 1][4]);
@@ -548,7 +522,6 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           // gate of this lane's token, spread to the lanes that hold it below
           float my_gate = 1.0f;
           if (MODE == kGateDown && !shared && tok < un.ntok) my_gate = __ldg(p.gate_perm + row);
-          if (leader && hh == 0 && j0 == 0) MOE_TRACE(MODE, i, 12);
           // The block (32 features = this quadrant's TMEM lanes, x 32 tokens =
           // columns j0..j0+31) in the m16n8 layout: lane half hf and column
           // group r give this thread features 16 hf + 8 e + lane / 4 (e = 0, 1)
@@ -585,8 +558,6 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
               }
             }
           }
-          const bool probe = leader && hh == 0 && j0 == 0;
-          if (probe) MOE_TRACE(MODE, i, 8);
           // Transpose into this warp's [32 tokens][32 features] tile, 64-byte
           // swizzled (16-byte chunk c of token row t sits at chunk c ^ ((t >> 1) & 3)),
           // with four transposing matrix stores: matrix m of store (hf, rp) is
@@ -610,8 +581,6 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           if (full_block) {
             fence_proxy_async_smem();
             __syncwarp();
-            if (probe) MOE_TRACE(MODE, i, 9);
-            if (probe) MOE_TRACE(MODE, i, 10);
             if (lane == 0) {
               tma_store_2d(shared ? &p.o_shared : &p.o_routed, tile, c0,
                            (int)(row_base + j0) + (shared ? p.out_row0_shared : 0));
@@ -619,21 +588,17 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
             }
           } else {
             __syncwarp();
-            if (probe) MOE_TRACE(MODE, i, 9);
             uint4 rowv[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c)
               rowv[c] = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(tile) + lane * 64 +
                                                         ((c ^ ((lane >> 1) & 3)) << 4));
-            if (probe) MOE_TRACE(MODE, i, 10);
             if (tok < un.ntok) store_row32(out_base + row * ld + c0, cols - c0, rowv);
           }
-          if (probe) MOE_TRACE(MODE, i, 11);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (leader) MOE_TRACE(MODE, i, 6);
       if (lane == 0) {
         for (int b = 0; b < 2; ++b)
           if ((mask >> b) & 1u) {
@@ -729,7 +694,7 @@ cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s, bool 
 }  // namespace
 
 cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStream_t s,
-                                   cudaEvent_t between, cudaEvent_t between2) {
+                                   cudaEvent_t between) {
   const int sms = device_sm_count();
   cudaError_t err0 = cudaMemsetAsync(a.sched, 0, 2 * sizeof(int), s);
   if (err0 != cudaSuccess) return err0;
@@ -768,7 +733,6 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   const int64_t units1 = chunks_bound * ((max_cols1 + kTcBN1 - 1) / kTcBN1);
   cudaError_t err = launch_one<kSwiGLU>(g1, (int)(units1 < sms ? units1 : sms), s, false);
   if (err == cudaSuccess && between) err = cudaEventRecord(between, s);
-  if (err == cudaSuccess && between2) err = cudaEventRecord(between2, s);
   if (err != cudaSuccess) return err;
 
   TcParams g2{};
@@ -800,18 +764,7 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   const int64_t units2 = chunks_bound * ((p.d + kTcBN2 - 1) / kTcBN2);
   // the down GEMM overlaps the SwiGLU GEMM's drain unless an event must be
   // recorded between the two
-  return launch_one<kGateDown>(g2, (int)(units2 < sms ? units2 : sms), s, !between && !between2);
+  return launch_one<kGateDown>(g2, (int)(units2 < sms ? units2 : sms), s, !between);
 }
 
 }  // namespace moe
-
-#ifdef MOE_UNIT_TRACE
-// Copies the unit trace ([2][kTraceCtas][kTraceUnits][16] u64) to host memory
-// and clears it (trace builds only).
-extern "C" MOE_API int moe_unit_trace_read(void* host_dst) {
-  cudaError_t e = cudaMemcpyFromSymbol(host_dst, moe::g_unit_trace, sizeof(moe::g_unit_trace));
-  if (e != cudaSuccess) return (int)e;
-  static unsigned long long zeros[2 * moe::kTraceCtas * moe::kTraceUnits * 16];
-  return (int)cudaMemcpyToSymbol(moe::g_unit_trace, zeros, sizeof(zeros));
-}
-#endif

@@ -40,7 +40,7 @@ struct Problem {
 struct Layout {
   size_t status, sched, logits, idx, gates, chunk_counts, chunk_base, counts, offsets;
   size_t grp_row0, grp_rows, unit_base1, unit_base2, perm, slot_pos, gate_perm;
-  size_t x_perm, h_perm, h_sh, y_rows, x_stage, y_stage;
+  size_t x_perm, h_perm, h_sh, y_rows, x_stage[2], y_stage;
   size_t total, total_host;
   int64_t n_chunks;
 };
@@ -75,25 +75,28 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
 bool make_tmap_bf16_swz(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                         uint32_t box_rows, int swizzle_bytes);
 
-// Router: logits (FP32 pipes) then selection. With router_scratch_bytes(p)
-// bytes of logits scratch the router uses router_k_splits(p) K ranges; with
-// less (at least T * N * 4) it uses as many as fit. `status` (may be null)
-// is reserved for MOE_DEV_* bits.
+// Router: logits (FP32 pipes) then selection. The reduction over d is cut
+// into S contiguous K ranges (S = `splits`, or router_k_splits(p) when
+// splits is 0) whose partial logits land in S planes of [T, N] fp32 in
+// `logits` (logits_bytes must cover them) and are added in a fixed order.
+// A token's logits depend only on its own row, d and S, so every S gives
+// deterministic bits and equal S gives equal bits at any T. `status` (may be
+// null) receives MOE_DEV_* bits.
 constexpr int kRouterTargetSms = 148;
 int router_k_splits(const Problem& p);
 size_t router_scratch_bytes(const Problem& p);
 cudaError_t launch_router(const Problem& p, const void* x, const void* W_r, const float* b,
                           float* logits, size_t logits_bytes, int32_t* idx, float* gates,
-                          unsigned* status, cudaStream_t s);
+                          unsigned* status, cudaStream_t s, int splits = 0);
 
 // Histogram / scan / scatter; bm, bn1, bn2 select the GEMM tile grid that
 // the unit tables describe.
 cudaError_t launch_dispatch(const Problem& p, const DispatchBuffers& db, int bm, int bn1, int bn2,
                             cudaStream_t s);
 
-// x_perm[r] = x[perm[r] / k]
-cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm,
-                          const int32_t* n_rows, void* x_perm, cudaStream_t s);
+// x_perm[slot_pos[t, s]] = x[t] for every placed (token, slot) pair
+cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* slot_pos, void* x_perm,
+                          cudaStream_t s);
 
 struct GemmArgs {
   const void* x;        // [T, d]
@@ -117,13 +120,14 @@ struct GemmArgs {
 };
 
 // Tensor-core (bf16) expert GEMMs: SwiGLU projection then gated down
-// projection; `between` and `between2` (optional) are recorded on s between
-// the two launches.
+// projection. `between` (optional) is recorded on s between the two
+// launches; without it the down projection is launched with programmatic
+// dependent launch and overlaps the SwiGLU GEMM's drain.
 cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStream_t s,
-                                   cudaEvent_t between, cudaEvent_t between2 = nullptr);
+                                   cudaEvent_t between);
 // fp32 SIMT expert GEMMs.
 cudaError_t launch_expert_gemms_simt(const Problem& p, const GemmArgs& a, cudaStream_t s,
-                                     cudaEvent_t between, cudaEvent_t between2 = nullptr);
+                                     cudaEvent_t between);
 
 // y[t] = sum over the token's rows slot_pos[t, 0..k) (ascending expert) of
 // y_rows, plus the shared row y_rows[R + t]

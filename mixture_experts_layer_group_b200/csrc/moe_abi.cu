@@ -120,7 +120,8 @@ Layout make_layout(const Problem& p) {
   L.h_sh = take((size_t)T * p.nsF * p.elem);
   L.y_rows = take((size_t)(R + T) * p.d * p.elem);
   L.total = off;
-  L.x_stage = take((size_t)T * p.d * p.elem);
+  L.x_stage[0] = take((size_t)T * p.d * p.elem);
+  L.x_stage[1] = take((size_t)T * p.d * p.elem);
   L.y_stage = take((size_t)T * p.d * p.elem);
   L.total_host = off;
   return L;
@@ -168,8 +169,7 @@ DispatchBuffers dispatch_buffers(const Layout& L, void* ws, const int32_t* idx, 
 moe_status forward_device(const Problem& p, const Layout& L, const void* x, const void* W_r,
                           const float* b, const void* W1, const void* W3, const void* W2,
                           const void* Ws1, const void* Ws3, const void* Ws2, void* y,
-                          int32_t* idx_out, float* gates_out, void* ws, cudaStream_t s,
-                          cudaEvent_t x_released = nullptr) {
+                          int32_t* idx_out, float* gates_out, void* ws, cudaStream_t s) {
   int32_t* idx = at<int32_t>(ws, L.idx);
   float* gates = at<float>(ws, L.gates);
   cudaError_t e0 = cudaMemsetAsync(at<void>(ws, L.status), 0, 4, s);
@@ -184,7 +184,7 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
                                   tc ? kTcBN2 : kSimtBN, s);
   if (e == cudaSuccess) e = mark_stage(2, s);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = launch_gather(p, x, db.perm, db.offsets + p.N, at<void>(ws, L.x_perm), s);
+  e = launch_gather(p, x, db.slot_pos, at<void>(ws, L.x_perm), s);
   if (e == cudaSuccess) e = mark_stage(3, s);
   if (e != cudaSuccess) return cuda_fail(e);
   GemmArgs ga;
@@ -206,9 +206,8 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
   ga.gate_perm = db.gate_perm;
   ga.status = db.status;
   ga.sched = at<int>(ws, L.sched);
-  // x is not read after the SwiGLU GEMM: x_released (optional) marks that point
-  e = tc ? launch_expert_gemms_tc(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr, x_released)
-         : launch_expert_gemms_simt(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr, x_released);
+  e = tc ? launch_expert_gemms_tc(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr)
+         : launch_expert_gemms_simt(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr);
   if (e == cudaSuccess) e = mark_stage(5, s);
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch_combine(p, ga.y_rows, db.slot_pos, y, s);
@@ -226,40 +225,72 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
 }
 
 // Per-workspace state of moe_forward_host: a non-blocking copy stream and
-// two events (no device memory), created on first use and kept for the
-// process lifetime.
+// a few events (no device memory), created on the workspace's first host
+// call and kept until moe_workspace_release(ws) or the process exits.
+//
+// x is staged in two slots that alternate between calls, so the input copy
+// of one call overlaps the whole of the previous call: the copy into a slot
+// waits only for the end of the call before last (which read that slot).
+// That holds while the workspace layout stays the same; a call with another
+// T or cfg (other offsets, which may overlap regions the previous call still
+// uses), or any device-buffer call on the workspace in between, makes the
+// copy wait for the end of the previous call instead.
 struct HostPipe {
   int device = -1;
   cudaStream_t copy = nullptr;
-  cudaEvent_t x_ready = nullptr;  // the staged x has landed
-  cudaEvent_t x_free = nullptr;   // the last call on this workspace no longer reads it
-  bool pending = false;           // x_free has been recorded
+  cudaEvent_t x_ready = nullptr;    // the staged x of the current call has landed
+  cudaEvent_t x_free[2] = {};       // the last call that used slot i no longer reads it
+  cudaEvent_t done = nullptr;       // end of the last call on this workspace (any entry point)
+  bool slot_used[2] = {false, false};
+  bool done_recorded = false;
+  bool relayout = true;             // next host call must wait for `done`
+  size_t stage_key[3] = {0, 0, 0};  // x slot offsets and bytes of the last host call
+  uint64_t calls = 0;
 };
 std::mutex g_pipe_mu;
 std::unordered_map<const void*, HostPipe> g_pipes;
 
-cudaError_t host_pipe(const void* ws, HostPipe** out) {
+void destroy_pipe(HostPipe& hp) {
+  if (hp.copy) cudaStreamDestroy(hp.copy);
+  if (hp.x_ready) cudaEventDestroy(hp.x_ready);
+  for (int i = 0; i < 2; ++i)
+    if (hp.x_free[i]) cudaEventDestroy(hp.x_free[i]);
+  if (hp.done) cudaEventDestroy(hp.done);
+  hp = HostPipe{};
+}
+
+cudaError_t host_pipe_locked(const void* ws, HostPipe** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(g_pipe_mu);
   HostPipe& hp = g_pipes[ws];
   if (hp.device != dev) {
-    if (hp.copy) {  // a different device reuses this address: start over
-      cudaStreamDestroy(hp.copy);
-      cudaEventDestroy(hp.x_ready);
-      cudaEventDestroy(hp.x_free);
-      hp = HostPipe{};
-    }
+    if (hp.copy) destroy_pipe(hp);  // a different device reuses this address: start over
     e = cudaStreamCreateWithFlags(&hp.copy, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.x_ready, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.x_free, cudaEventDisableTiming);
-    if (e != cudaSuccess) return e;
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&hp.x_free[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      destroy_pipe(hp);
+      return e;
+    }
     hp.device = dev;
-    hp.pending = false;
   }
   *out = &hp;
   return cudaSuccess;
+}
+
+// A device-buffer entry point (moe_route, moe_dispatch, moe_forward) has
+// enqueued work on `s` that uses ws: if moe_forward_host has state for this
+// workspace, mark the end of that work so the next host call's input copy
+// waits for it (the copy runs on another stream).
+cudaError_t note_device_use(const void* ws, cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  auto it = g_pipes.find(ws);
+  if (it == g_pipes.end() || !it->second.done) return cudaSuccess;
+  it->second.relayout = true;
+  it->second.done_recorded = true;
+  return cudaEventRecord(it->second.done, s);
 }
 
 moe_status check_weights(const Problem& p, const void* W_r, const float* b, const void* W1,
@@ -309,7 +340,11 @@ moe_status moe_route(const moe_cfg* cfg, int64_t T, const void* x, const void* W
   if (!x || !W_r || !topk_idx || !gates || !aligned16(x) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
   Layout L = make_layout(p);
   if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
-  return run_router(p, L, x, W_r, b, topk_idx, gates, ws, (cudaStream_t)stream);
+  cudaError_t e = cudaMemsetAsync(at<void>(ws, L.status), 0, 4, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if ((st = run_router(p, L, x, W_r, b, topk_idx, gates, ws, (cudaStream_t)stream)) != MOE_OK) return st;
+  if ((e = note_device_use(ws, (cudaStream_t)stream)) != cudaSuccess) return cuda_fail(e);
+  return MOE_OK;
 }
 
 moe_status moe_dispatch(const moe_cfg* cfg, int64_t T, const int32_t* topk_idx, int32_t* counts,
@@ -336,6 +371,7 @@ moe_status moe_dispatch(const moe_cfg* cfg, int64_t T, const int32_t* topk_idx, 
     return cuda_fail(e);
   if (perm && (e = cudaMemcpyAsync(perm, db.perm, (size_t)p.R * 4, cudaMemcpyDeviceToDevice, s)))
     return cuda_fail(e);
+  if ((e = note_device_use(ws, s)) != cudaSuccess) return cuda_fail(e);
   return MOE_OK;
 }
 
@@ -351,8 +387,11 @@ moe_status moe_forward(const moe_cfg* cfg, int64_t T, const void* x, const void*
   if ((st = check_weights(p, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2)) != MOE_OK) return st;
   Layout L = make_layout(p);
   if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
-  return forward_device(p, L, x, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y, topk_idx_out, gates_out, ws,
-                        (cudaStream_t)stream);
+  st = forward_device(p, L, x, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y, topk_idx_out, gates_out, ws,
+                      (cudaStream_t)stream);
+  if (st != MOE_OK) return st;
+  cudaError_t e = note_device_use(ws, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
 moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
@@ -369,24 +408,53 @@ moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, c
   if ((st = check_ws(L, ws, ws_bytes, L.total_host)) != MOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const size_t bytes = (size_t)p.T * p.d * p.elem;
-  void* xd = at<void>(ws, L.x_stage);
   void* yd = at<void>(ws, L.y_stage);
-  // The host-to-device copy runs on the workspace's own copy stream, after
-  // the previous call on this workspace released the staged x (end of its
-  // SwiGLU GEMM): consecutive calls overlap this copy with the previous
-  // call's down projection, combine and device-to-host copy.
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
   HostPipe* hp = nullptr;
-  cudaError_t e = host_pipe(ws, &hp);
-  if (e == cudaSuccess && hp->pending) e = cudaStreamWaitEvent(hp->copy, hp->x_free, 0);
+  cudaError_t e = host_pipe_locked(ws, &hp);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const size_t key[3] = {L.x_stage[0], L.x_stage[1], bytes};
+  if (std::memcmp(key, hp->stage_key, sizeof(key)) != 0) hp->relayout = true;
+  if (hp->relayout) {
+    // another layout (or device work) since the last host call: the copy may
+    // land on regions the previous call still uses, so wait for all of it
+    hp->slot_used[0] = hp->slot_used[1] = false;
+    if (hp->done_recorded) e = cudaStreamWaitEvent(hp->copy, hp->done, 0);
+    hp->calls = 0;
+  }
+  const int slot = (int)(hp->calls & 1u);
+  void* xd = at<void>(ws, L.x_stage[slot]);
+  if (e == cudaSuccess && hp->slot_used[slot]) e = cudaStreamWaitEvent(hp->copy, hp->x_free[slot], 0);
   if (e == cudaSuccess) e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, hp->copy);
   if (e == cudaSuccess) e = cudaEventRecord(hp->x_ready, hp->copy);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->x_ready, 0);
   if (e != cudaSuccess) return cuda_fail(e);
-  st = forward_device(p, L, xd, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, yd, nullptr, nullptr, ws, s, hp->x_free);
+  st = forward_device(p, L, xd, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, yd, nullptr, nullptr, ws, s);
   if (st != MOE_OK) return st;
-  hp->pending = true;
+  // the slot is free again once this call's kernels are done
+  if ((e = cudaEventRecord(hp->x_free[slot], s)) != cudaSuccess) return cuda_fail(e);
+  hp->slot_used[slot] = true;
   e = cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaEventRecord(hp->done, s);
   if (e != cudaSuccess) return cuda_fail(e);
+  hp->done_recorded = true;
+  hp->relayout = false;
+  std::memcpy(hp->stage_key, key, sizeof(key));
+  ++hp->calls;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_release(const void* ws) {
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  auto it = g_pipes.find(ws);
+  if (it == g_pipes.end()) return MOE_OK;
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e == cudaSuccess && it->second.device >= 0 && cur != it->second.device) e = cudaSetDevice(it->second.device);
+  if (e != cudaSuccess) return cuda_fail(e);
+  destroy_pipe(it->second);
+  g_pipes.erase(it);
+  if (cur >= 0) cudaSetDevice(cur);
   return MOE_OK;
 }
 

@@ -16,8 +16,11 @@
 namespace moe {
 namespace {
 
-// Largest scratch a call may use: the router's fp32 logits, T * n_routed * 4
-// bytes (the router splits its reduction only as far as the array allows).
+// Size of the fixed scratch array. A call needs T * n_routed * 4 bytes of it
+// at least (one plane of fp32 logits for every token); a call that needs
+// more planes than fit (moe_route splits the reduction over d into S ranges,
+// one plane each) runs the router over slices of the tokens in turn, each
+// slice with the same S, so the logits are bitwise those of moe_route.
 constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB
 
 __device__ __align__(256) unsigned char g_route_scratch[kNoallocScratchBytes];
@@ -61,11 +64,24 @@ extern "C" moe_status moe_route_noalloc(const moe_cfg* cfg, int64_t T, const voi
   if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(W_r) & 15u))
     return MOE_ERR_INVALID_ARG;
   if ((size_t)T * (size_t)p.N * sizeof(float) > kNoallocScratchBytes) return MOE_ERR_UNSUPPORTED;
+  // moe_route's split count for the whole batch, and the largest token slice
+  // whose S planes fit the array (a multiple of 64 tokens, the router's tile
+  // height; at least 256 tokens since S <= 16 and n_routed <= 512)
+  const int S = router_k_splits(p);
+  int64_t slice = (int64_t)(kNoallocScratchBytes / ((size_t)S * (size_t)p.N * sizeof(float)));
+  if (slice < T) slice = slice / 64 * 64;
+  if (slice < 1) return MOE_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   cudaError_t e = scratch_address(&scratch);
-  if (e == cudaSuccess)
-    e = launch_router(p, x, W_r, b, static_cast<float*>(scratch), kNoallocScratchBytes, topk_idx, gates,
-                      nullptr, static_cast<cudaStream_t>(stream));
+  const uint8_t* xb = static_cast<const uint8_t*>(x);
+  for (int64_t t0 = 0; e == cudaSuccess && t0 < T; t0 += slice) {
+    Problem ps = p;  // the same layer on tokens [t0, t0 + slice)
+    ps.T = T - t0 < slice ? T - t0 : slice;
+    ps.R = ps.T * p.k;
+    e = launch_router(ps, xb + t0 * (int64_t)p.d * p.elem, W_r, b, static_cast<float*>(scratch),
+                      kNoallocScratchBytes, topk_idx + t0 * p.k, gates + t0 * p.k, nullptr,
+                      static_cast<cudaStream_t>(stream), S);
+  }
   if (e != cudaSuccess) {
     record_cuda_error(e);
     return MOE_ERR_CUDA;

@@ -240,6 +240,7 @@ struct SelectArgs {
   float route_scale;
   int32_t* idx;
   float* gates;
+  unsigned* status;     // MOE_DEV_* bits (may be null)
 };
 
 // One warp per token. Lane l holds experts e = 32 j + l, j < V.
@@ -281,11 +282,26 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
 #pragma unroll
     for (int j = 0; j < V; ++j) s[j] = (32 * j + lane < N) ? 1.0f / (1.0f + expf(-s[j])) : 0.f;
   }
+  // A NaN or infinite logit or key (from non-finite x, W_r or b) is
+  // recorded in the status word; its key is replaced by the lowest finite
+  // value, so the token still gets k distinct experts below N (which ones is
+  // then arbitrary) and every other token is unaffected.
+  bool bad = false;
 #pragma unroll
   for (int j = 0; j < V; ++j) {
     int e = 32 * j + lane;
-    key[j] = e < N ? s[j] + (a.bias ? a.bias[e] : 0.f) : -INFINITY;
+    if (e < N) {
+      float kv = s[j] + (a.bias ? a.bias[e] : 0.f);
+      if (!isfinite(kv) || !isfinite(s[j])) {
+        bad = true;
+        if (kv != kv) kv = -FLT_MAX;
+      }
+      key[j] = kv;
+    } else {
+      key[j] = -INFINITY;
+    }
   }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, MOE_DEV_NONFINITE);
 
   if (a.G > 1) {
     // group scores: lane g keeps the score of group g (G <= 32)
@@ -306,13 +322,15 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
         merge_top2(t1, t2, o1, o2);
       }
       float gsc = a.group_score == MOE_GROUP_MAX ? t1 : t1 + t2;
+      if (gsc != gsc) gsc = -FLT_MAX;  // +inf + -inf keys of a non-finite token
       if (lane == g) my_gs = gsc;
     }
     uint32_t allowed = 0;
+    bool g_taken = lane >= a.G;  // lane g: group g already kept (or no such group)
     for (int r = 0; r < a.TG; ++r) {
-      Cand c = warp_best(Cand{lane < a.G ? my_gs : -INFINITY, lane < a.G ? lane : 1 << 30});
+      Cand c = warp_best(Cand{g_taken ? -INFINITY : my_gs, g_taken ? 1 << 30 : lane});
       allowed |= 1u << (c.e & 31);
-      if (lane == c.e) my_gs = -INFINITY;
+      if (lane == c.e) g_taken = true;
     }
 #pragma unroll
     for (int j = 0; j < V; ++j)
@@ -321,12 +339,13 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
 
   int sel_e = 0;
   float sel_s = 0.f, ssum = 0.f;
+  uint32_t taken = 0;  // bit j: this lane's expert 32 j + lane is already selected
   for (int slot = 0; slot < a.k; ++slot) {
     Cand c{-INFINITY, 1 << 30};
 #pragma unroll
     for (int j = 0; j < V; ++j) {
       int e = 32 * j + lane;
-      if (e < N && better(key[j], e, c.v, c.e)) c = Cand{key[j], e};
+      if (e < N && !((taken >> j) & 1u) && better(key[j], e, c.v, c.e)) c = Cand{key[j], e};
     }
     c = warp_best(c);
     int owner = c.e & 31, jj = c.e >> 5;
@@ -335,7 +354,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
     for (int j = 0; j < V; ++j)
       if (lane == owner && j == jj) {
         sv = s[j];
-        key[j] = -INFINITY;
+        taken |= 1u << j;
       }
     sv = __shfl_sync(0xffffffffu, sv, owner);
     ssum += sv;
@@ -380,13 +399,12 @@ size_t router_scratch_bytes(const Problem& p) {
 
 cudaError_t launch_router(const Problem& p, const void* x, const void* W_r, const float* b,
                           float* logits, size_t logits_bytes, int32_t* idx, float* gates,
-                          unsigned* status, cudaStream_t s) {
-  (void)status;
-  // as many K splits as router_k_splits(p) asks for and the scratch can hold
+                          unsigned* status, cudaStream_t s, int splits) {
+  // K splits: `splits` when given, else router_k_splits(p); the scratch must
+  // hold one [T, N] plane of partial logits per split
   const size_t plane = (size_t)p.T * (size_t)p.N * sizeof(float);
-  int S = router_k_splits(p);
-  if ((size_t)S * plane > logits_bytes) S = (int)(logits_bytes / plane);
-  if (S < 1) return cudaErrorInvalidValue;
+  const int S = splits > 0 ? splits : router_k_splits(p);
+  if (S > 16 || (size_t)S * plane > logits_bytes) return cudaErrorInvalidValue;
   const int k_len = ((p.d + S - 1) / S + kLBK - 1) / kLBK * kLBK;
   dim3 grid((unsigned)((p.N + kLBN - 1) / kLBN), (unsigned)((p.T + kLBT - 1) / kLBT), (unsigned)S);
   static std::mutex mu;
@@ -417,7 +435,7 @@ cudaError_t launch_router(const Problem& p, const void* x, const void* W_r, cons
   if (err != cudaSuccess) return err;
 
   SelectArgs a{logits, S, b, p.T, p.N, p.k, p.G, p.TG, p.score_fn, p.group_score, p.normalize,
-               p.route_scale, idx, gates};
+               p.route_scale, idx, gates, status};
   const int warps = 8;
   unsigned blocks = (unsigned)((p.T + warps - 1) / warps);
   int V = (p.N + 31) / 32;

@@ -4,13 +4,19 @@
 // and returns instead of hanging. This entry point makes one such wait run
 // out on purpose -- an mbarrier that nothing ever completes -- without any
 // fault, trap or unbounded loop.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 namespace {
 
+// One status word per device, shared by every call: calls are serialised by
+// g_selftest_mu (each call synchronises its stream before it returns), so no
+// two calls in this process ever touch the word at the same time.
 __device__ unsigned g_selftest_status;
+std::mutex g_selftest_mu;
 
 __global__ void wait_timeout_probe(unsigned* status) {
   __shared__ __align__(8) uint64_t bar;
@@ -33,6 +39,7 @@ using namespace moe;
 extern "C" moe_status moe_selftest_wait_timeout(uint32_t* bits, void* stream) {
   if (!bits) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_selftest_mu);
   void* status = nullptr;
   cudaError_t e = cudaGetSymbolAddress(&status, g_selftest_status);
   if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, sizeof(unsigned), s);

@@ -6,11 +6,20 @@ Comparison rules:
     oracle does not flag; a flagged token (selection margin < 1e-6) may pick
     any selection that is optimal within the margin. Slot order may differ
     only where the oracle flags an order tie.
-  * outputs: max relative Frobenius error ||y - y_ref|| / ||y_ref|| within
-    2e-2 for bf16 layers and 1e-5 for fp32 layers, where y_ref is the oracle
-    evaluated with the GPU's selection for flagged tokens.
+  * outputs: the relative Frobenius error ||y - y_ref|| / ||y_ref|| over the
+    checked rows within 2e-2 for bf16 layers and 1e-5 for fp32 layers, and
+    the same error of every single token row, max_t ||y_t - ref_t|| /
+    ||ref_t||, within 1e-2 (bf16) and 1e-5 (fp32), where y_ref is the oracle
+    evaluated with the GPU's selection for flagged tokens. The bf16 bound per
+    token: the path rounds h, each gated expert row and y to bf16 (relative
+    RMS 2^-9 / sqrt(3) ~ 1.1e-3 each), so a token's row error is ~2-3e-3
+    with d in the hundreds or more; 1e-2 leaves a factor of 3 or more, while
+    a token row that is wrong in a quarter of its columns shows ~0.5.
 """
 from __future__ import annotations
+
+import concurrent.futures
+import threading
 
 import numpy as np
 import torch
@@ -21,6 +30,7 @@ from moe_inputs import device as mdev
 import mixture_experts_layer_group_b200 as moe
 
 TOL = {"bf16": 2e-2, "f32": 1e-5}
+TOKEN_TOL = {"bf16": 1e-2, "f32": 1e-5}
 
 
 def cfg_of(s: mi.LayerShape) -> moe.MoeCfg:
@@ -101,6 +111,25 @@ def rel_fro(y, ref):
     return float(np.linalg.norm(y - ref) / max(np.linalg.norm(ref), 1e-300))
 
 
+def token_rel_max(y, ref):
+    """max over token rows of ||y_t - ref_t|| / ||ref_t||, and the worst row."""
+    num = np.linalg.norm(y - ref, axis=1)
+    den = np.maximum(np.linalg.norm(ref, axis=1), 1e-300)
+    r = num / den
+    t = int(np.argmax(r)) if r.size else -1
+    return (float(r[t]) if r.size else 0.0), t
+
+
+def check_outputs(y, ref, dtype, what=""):
+    """Whole-block relative Frobenius error and the worst token row, each
+    within its bound; returns (whole, worst_token, worst_row)."""
+    err = rel_fro(y, ref)
+    tok, t = token_rel_max(y, ref)
+    assert err <= TOL[dtype], (what, "rel_fro", err)
+    assert tok <= TOKEN_TOL[dtype], (what, "token", t, tok)
+    return err, tok, t
+
+
 def oracle_forward(s: mi.LayerShape, x64, W_r64, b, expert_fn, shared, gidx=None):
     """fp64 oracle output for token rows x64; tokens the oracle flags are
     re-evaluated with the GPU's selection gidx (when given)."""
@@ -122,6 +151,61 @@ def host_expert_fn(s: mi.LayerShape):
         w1, w3, w2 = mi.host_expert(s, e)
         return f64(w1), f64(w3), f64(w2)
     return fn
+
+
+class PrefetchedExperts:
+    """expert(e) for the oracle, with the fp64 weights of the next experts in
+    `order` generated and widened on worker threads (at most `depth` ahead,
+    so only a few experts are resident). Experts outside the order, or asked
+    for again, are built on the spot."""
+
+    def __init__(self, s: mi.LayerShape, order, depth: int = 6):
+        self.fn = host_expert_fn(s)
+        self.order = list(order)
+        self.pos = {e: i for i, e in enumerate(self.order)}
+        self.pool = concurrent.futures.ThreadPoolExecutor(max_workers=depth)
+        self.depth = depth
+        self.futs = {}
+        self.next = 0
+        self.lock = threading.Lock()
+        self._fill(0)
+
+    def _fill(self, i):
+        with self.lock:
+            self.next = max(self.next, i)
+            while self.next < len(self.order) and self.next < i + self.depth:
+                e = self.order[self.next]
+                self.futs[e] = self.pool.submit(self.fn, e)
+                self.next += 1
+
+    def __call__(self, e):
+        fut = self.futs.pop(e, None)
+        if e in self.pos:
+            self._fill(self.pos[e] + 1)
+        return fut.result() if fut is not None else self.fn(e)
+
+    def close(self):
+        self.pool.shutdown(wait=True, cancel_futures=True)
+
+
+def chunk_probe_rows(idx: np.ndarray, n_routed: int, max_tok: int = 256):
+    """Token rows that reach the expert GEMMs' chunk edges: for every routed
+    expert, the first token of each chunk the kernels cut its rows into
+    (ceil(rows / max_tok) chunks of equal size) and its last token (the end
+    of its last, ragged 32-token block)."""
+    T, k = idx.shape
+    picks = set()
+    for e in range(n_routed):
+        toks = np.nonzero((idx == e).any(axis=1))[0]
+        n = toks.size
+        if n == 0:
+            continue
+        nc = (n + max_tok - 1) // max_tok
+        cs = (n + nc - 1) // nc
+        for c in range(nc):
+            picks.add(int(toks[c * cs]))
+        picks.add(int(toks[-1]))
+    return np.array(sorted(picks), dtype=np.int64)
 
 
 def host_shared64(s: mi.LayerShape):

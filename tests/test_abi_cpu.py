@@ -123,3 +123,12 @@ def test_argument_errors_need_no_device(L):
     assert L.moe_bias_update(ctypes.byref(cfg), 4, fake, ctypes.c_float(float("nan")), fake, None) == 1
     assert L.moe_bias_update(None, 4, fake, ctypes.c_float(1e-3), fake, None) == 1
     assert L.moe_last_cuda_error() == 0
+
+
+def test_make_cfg_rejects_unknown_strings():
+    # a misspelt score, group score or dtype is an error, not a silent default
+    for kw in ({"score": "sigmoidd"}, {"group_score": "top2"}, {"dtype": "fp16"}):
+        with pytest.raises(ValueError):
+            moe.make_cfg(64, 64, 8, 0, 2, **kw)
+    c = moe.make_cfg(64, 64, 8, 0, 2, score="sigmoid", group_score="max", dtype="f32")
+    assert (c.score_fn, c.group_score, c.dtype) == (moe.MOE_SIGMOID, moe.MOE_GROUP_MAX, moe.MOE_F32)

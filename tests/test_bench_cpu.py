@@ -12,25 +12,27 @@ import moe_inputs as mi
 def test_algorithmic_counts_v3_prefill():
     s = mi.SHAPES["v3_prefill_bf16"]
     counts = np.full(s.n_routed, s.T * s.top_k // s.n_routed)  # every expert touched
-    U, flops, layer_bytes, swiglu_bytes = bench.algorithmic(s, counts)
-    assert U == 256
+    A = bench.algorithmic(s, counts)
+    assert A["U"] == 256
     # T (k + n_s) 6 d d_ff (the benchmark spec's count)
-    assert flops == 4096 * 9 * 6 * 7168 * 2048
+    assert A["flops"] == 4096 * 9 * 6 * 7168 * 2048
     # touched expert weights (3 matrices of d x d_ff per expert, bf16) + router + x in + y out
-    assert layer_bytes == 257 * 3 * 7168 * 2048 * 2 + 256 * 7168 * 2 + 2 * 4096 * 7168 * 2
+    assert A["layer_bytes"] == 257 * 3 * 7168 * 2048 * 2 + 256 * 7168 * 2 + 2 * 4096 * 7168 * 2
     assert abs(257 * 3 * 7168 * 2048 * 2 / 1e9 - 22.64) < 0.01  # the 22.6 GB of weights the bench states
-    # SwiGLU GEMM: W1, W3 of touched experts + shared, token rows read, h written
+    # SwiGLU GEMM, algorithmic: W1, W3 of touched experts + shared, x read once
+    assert A["swiglu_alg"] == 257 * 2 * 7168 * 2048 * 2 + 4096 * 7168 * 2
+    # and with the implementation's token-row reads and h writes
     R = 4096 * 8
-    assert swiglu_bytes == 257 * 2 * 7168 * 2048 * 2 + (R + 4096) * 7168 * 2 + (R + 4096) * 2048 * 2
+    assert A["swiglu_impl"] == 257 * 2 * 7168 * 2048 * 2 + (R + 4096) * 7168 * 2 + (R + 4096) * 2048 * 2
 
 
 def test_untouched_experts_do_not_count():
     s = mi.SHAPES["v3_decode_bf16"]
     counts = np.zeros(s.n_routed, dtype=np.int64)
     counts[:57] = 1
-    U, _, layer_bytes, _ = bench.algorithmic(s, counts)
-    assert U == 57
-    assert layer_bytes == 58 * 3 * 7168 * 2048 * 2 + 256 * 7168 * 2 + 2 * 128 * 7168 * 2
+    A = bench.algorithmic(s, counts)
+    assert A["U"] == 57
+    assert A["layer_bytes"] == 58 * 3 * 7168 * 2048 * 2 + 256 * 7168 * 2 + 2 * 128 * 7168 * 2
 
 
 def test_sample_token_cap_bounds():

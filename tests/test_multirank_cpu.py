@@ -96,3 +96,20 @@ def test_reference_arm_reports_on_rank0_only():
         p.join(timeout=60)
     assert got[0][0] == 0 and got[1][0] == 0
     assert '"impl": "reference"' in got[0][1] and got[1][1].strip() == ""
+
+
+def test_bench_gpus_2_starts_two_ranks():
+    # `bench.py --gpus 2` outside torchrun re-launches itself as two local
+    # ranks; --check-launch stops after the ranks have joined a gloo group
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--check-launch"],
+                         capture_output=True, text=True, timeout=240, env=env, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    rep = json.loads([ln for ln in out.stdout.splitlines() if ln.startswith("{")][-1])
+    assert rep["n_gpus"] == 2
+    assert sorted(r["rank"] for r in rep["ranks"]) == [0, 1]
+    assert len({r["pid"] for r in rep["ranks"]}) == 2

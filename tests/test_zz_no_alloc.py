@@ -56,6 +56,28 @@ def test_route_noalloc_matches_route_on_consecutive_calls():
         np.testing.assert_allclose(gates.cpu().numpy(), ref_gates.cpu().numpy(), rtol=GATE_RTOL, atol=1e-7)
 
 
+def test_route_noalloc_matches_route_bitwise_at_v3_prefill_size():
+    # T = 4096 at the V3 shape: moe_route's partial logits for the whole batch
+    # (8 K ranges x 4 MiB) do not fit the fixed 8 MiB array, so the call runs
+    # the router over token slices with moe_route's K ranges; indices and
+    # gates must be moe_route's bit for bit, on two calls in a row
+    from mixture_experts_layer_group_b200 import build
+    from moe_inputs import build as gen_build
+    gen_build.build()
+    build.build()
+    torch.cuda.set_device(0)
+    s = mi.SHAPES["v3_prefill_bf16"]
+    cfg = _cfg(s)
+    w = {"W_r": mdev.device_tensor(s, "W_r"), "b": mdev.device_tensor(s, "b")}
+    x = mdev.device_tensor(s, "x")
+    ref_idx, ref_gates = _route_with_workspace(s, cfg, x, w)
+    for _ in range(2):
+        idx, gates = _route_noalloc(s, cfg, x, w)
+        torch.cuda.synchronize()
+        assert torch.equal(idx, ref_idx)
+        assert torch.equal(gates, ref_gates)
+
+
 def test_route_noalloc_rejects_sizes_beyond_its_scratch():
     torch.cuda.set_device(0)
     s = mi.SHAPES["v3_prefill_bf16"].with_(T=8193)  # 8193 * 256 * 4 bytes > 8 MiB
