@@ -170,6 +170,13 @@ def max_over_ranks(values, device=None):
     return t.tolist()
 
 
+def weight_bytes_per_element(s: mi.LayerShape) -> float:
+    """HBM bytes per expert-weight element: 2 (bf16), 4 (fp32), or 1 + 1/128^2 (e4m3 + block scale)."""
+    if s.wdtype == "fp8":
+        return 1.0 + 1.0 / (128 * 128)
+    return 2.0 if s.dtype == "bf16" else 4.0
+
+
 def algorithmic(s: mi.LayerShape, counts: np.ndarray):
     """What the layer must do, independent of how: FLOPs of the expert
     matmuls, HBM bytes of the layer (touched expert weights, router weights,
@@ -178,10 +185,11 @@ def algorithmic(s: mi.LayerShape, counts: np.ndarray):
     plus the implementation's own token-row reads and SwiGLU-row writes."""
     U = int((counts > 0).sum())
     e = 2 if s.dtype == "bf16" else 4
+    we = weight_bytes_per_element(s)
     flops = s.T * (s.top_k + s.n_shared) * 6 * s.d * s.d_ff
-    layer_bytes = (U + s.n_shared) * 3 * s.d * s.d_ff * e + s.n_routed * s.d * e + 2 * s.T * s.d * e
+    layer_bytes = int((U + s.n_shared) * 3 * s.d * s.d_ff * we) + s.n_routed * s.d * e + 2 * s.T * s.d * e
     R = s.T * s.top_k
-    w13 = (U + s.n_shared) * 2 * s.d * s.d_ff * e
+    w13 = int((U + s.n_shared) * 2 * s.d * s.d_ff * we)
     swiglu_alg = w13 + s.T * s.d * e
     swiglu_impl = (w13 + (R + (s.T if s.n_shared else 0)) * s.d * e
                    + (R * s.d_ff + s.T * s.n_shared * s.d_ff) * e)
@@ -209,15 +217,19 @@ class Layer:
         w = self.w
         self.wargs = (w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"])
 
+    def _forward(self, *extra):
+        fwd = self.moe.forward_fp8 if self.s.wdtype == "fp8" else self.moe.forward
+        fwd(self.cfg, self.s.T, self.x, *self.wargs, self.y, self.ws, *extra, stream=self.stream)
+
     def step(self):
-        self.moe.forward(self.cfg, self.s.T, self.x, *self.wargs, self.y, self.ws, stream=self.stream)
+        self._forward()
 
     def routing_counts(self):
         import torch
         s = self.s
         idx = torch.empty((s.T, s.top_k), dtype=torch.int32, device="cuda")
         gates = torch.empty((s.T, s.top_k), dtype=torch.float32, device="cuda")
-        self.moe.forward(self.cfg, s.T, self.x, *self.wargs, self.y, self.ws, idx, gates, stream=self.stream)
+        self._forward(idx, gates)
         torch.cuda.synchronize()
         status = self.moe.device_status(self.cfg, s.T, self.ws)
         return np.bincount(idx.cpu().numpy().reshape(-1), minlength=s.n_routed), status
@@ -330,7 +342,23 @@ def run_ours(args, rank, world, local_rank):
         D.free()
         dec = (ds, dms, dcounts, dstatus, dstage, dclk.summary())
 
-    vals = [ms, e2e_ms] + ([dec[1]] if dec else [])
+    # --- the V3 prefill layer with FP8 expert weights, timed the same way
+    f8 = None
+    if not args.no_fp8 and s.name == "v3_prefill_bf16":
+        fs = mi.SHAPES["v3_prefill_fp8"]
+        Fl = Layer(fs, rank)
+        for _ in range(args.warmup):
+            Fl.step()
+        fcounts, fstatus = Fl.routing_counts()
+        if world > 1:
+            dist.barrier()
+        with ClockSampler(uuid) as fclk:
+            fms = Fl.timed(args.steps)
+        fstage = Fl.stage_pass(min(args.steps, 20))
+        Fl.free()
+        f8 = (fs, fms, fcounts, fstatus, fstage, fclk.summary())
+
+    vals = [ms, e2e_ms] + ([dec[1]] if dec else []) + ([f8[1]] if f8 else [])
     vals = max_over_ranks(vals, device="cuda")
     ms, e2e_ms = vals[0], vals[1]
     if rank != 0:
@@ -402,6 +430,22 @@ def run_ours(args, rank, world, local_rank):
                          "bound": "hbm" if d_t_hbm > d_t_tc else "tensor",
                          "bytes": DA["layer_bytes"], "stage_ms": {k: round(v, 4) for k, v in dstage.items()},
                          "clocks": dclocks, "device_status": dstatus}
+    if f8:
+        fs, fms, fcounts, fstatus, fstage, fclocks = f8
+        fms = vals[-1]
+        FA = algorithmic(fs, fcounts)
+        ft = fms / 1e3
+        f_t_hbm = FA["layer_bytes"] / (peaks["hbm_gbs"] * 1e9)
+        f_t_tc = FA["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+        out["fp8"] = {"workload": describe(fs) + ", expert weights e4m3 with one power-of-two scale per 128x128 block",
+                      "ms_per_step": round(fms, 4), "tokens_per_s": round(world * fs.T / ft, 1),
+                      "hbm_gbs": round(FA["layer_bytes"] / ft / 1e9, 1),
+                      "hbm_frac": round(FA["layer_bytes"] / ft / 1e9 / peaks["hbm_gbs"], 4),
+                      "tflops": round(FA["flops"] / ft / 1e12, 1),
+                      "binding_frac": round(max(f_t_hbm, f_t_tc) / ft, 4),
+                      "bound": "hbm" if f_t_hbm > f_t_tc else "tensor (bf16 MMA after dequantisation)",
+                      "bytes": FA["layer_bytes"], "stage_ms": {k: round(v, 4) for k, v in fstage.items()},
+                      "clocks": fclocks, "device_status": fstatus}
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(s, args.cpu_tokens)
     return out
@@ -596,6 +640,7 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the V3 decode sub-measurement")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-weight V3 prefill sub-measurement")
     ap.add_argument("--check-launch", action="store_true",
                     help="start the ranks, join a gloo process group, report them and exit (no GPU work)")
     ap.add_argument("--stage", default="layer", choices=["layer", "router", "bias"],

@@ -170,6 +170,44 @@ MOE_API moe_status moe_forward(const moe_cfg* cfg, int64_t T, const void* x, con
                        float* gates_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * One expert weight matrix in FP8: e4m3 codes with one power-of-two scale
+ * per 128 x 128 block, the block-scaled FP8 layout of DeepSeek-V3-style
+ * checkpoints (the "DeepSeek-V3.2-Exp · Mixture of experts" page, Parameters:
+ * the checkpoint carries FP8 block scales). Element (r, c) has the value
+ *   e4m3(codes[r * cols + c]) * 2^(scales[(r / 128) * (cols / 128) + c / 128] - 127)
+ * with e4m3 the OCP FP8 E4M3 format (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits, no infinities, 0x7F / 0xFF NaN, largest finite 448) and the
+ * scale byte a UE8M0 exponent.
+ *   codes   [rows, cols] uint8, row-major, 16-byte aligned
+ *   scales  [rows / 128, cols / 128] uint8
+ * For the routed experts the matrices are stacked as in moe_forward (W1, W3:
+ * rows = n_routed * d_ff, cols = d; W2: rows = n_routed * d, cols = d_ff).
+ */
+typedef struct moe_fp8_matrix {
+  const void* codes;
+  const uint8_t* scales;
+} moe_fp8_matrix;
+
+/*
+ * moe_forward with FP8 expert weights (routed and shared): the same layer,
+ * tokens, router (W_r bf16), outputs and workspace as moe_forward with
+ * cfg->dtype == MOE_BF16. Each weight tile is dequantised exactly to bf16 in
+ * shared memory (a power-of-two scale times an e4m3 value is a bf16 value)
+ * and multiplied on the tensor cores as in the bf16 path, so the result
+ * equals moe_forward run on the dequantised weights (bit for bit, as long as
+ * every dequantised weight is a normal bf16 number). Weight bytes streamed
+ * from HBM are halved.
+ * Requires d, d_ff and n_shared * d_ff to be multiples of 128 and at most
+ * 8192 (MOE_ERR_UNSUPPORTED otherwise) and cfg->dtype == MOE_BF16
+ * (MOE_ERR_INVALID_ARG otherwise). Ws1 / Ws3 / Ws2 are NULL iff n_shared == 0.
+ */
+MOE_API moe_status moe_forward_fp8(const moe_cfg* cfg, int64_t T, const void* x, const void* W_r, const float* b,
+                                   const moe_fp8_matrix* W1, const moe_fp8_matrix* W3, const moe_fp8_matrix* W2,
+                                   const moe_fp8_matrix* Ws1, const moe_fp8_matrix* Ws3,
+                                   const moe_fp8_matrix* Ws2, void* y, int32_t* topk_idx_out, float* gates_out,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/*
  * moe_forward with the token rows in host memory: copies x_host [T, d] to
  * the device inside the workspace, runs the layer, and copies y back to
  * y_host [T, d], all enqueued on `stream`. Host buffers should be pinned

@@ -22,6 +22,7 @@ MOE_DEV_WAIT_TIMEOUT, MOE_DEV_BAD_EXPERT, MOE_DEV_DUP_EXPERT, MOE_DEV_TMEM_ALLOC
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE"}
 EXPORTS = ["moe_workspace_size", "moe_workspace_size_host", "moe_route", "moe_dispatch", "moe_forward",
+           "moe_forward_fp8",
            "moe_forward_host", "moe_workspace_release", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update", "moe_selftest_wait_timeout",
            "moe_status_string", "moe_last_cuda_error"]
 STAGES = ["router", "dispatch", "gather", "gemm_swiglu", "gemm_gate", "combine"]
@@ -35,6 +36,12 @@ class MoeCfg(ctypes.Structure):
                 ("topk_groups", ctypes.c_int32), ("score_fn", ctypes.c_int32),
                 ("normalize", ctypes.c_int32), ("route_scale", ctypes.c_float),
                 ("group_score", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class Fp8Matrix(ctypes.Structure):
+    """moe_fp8_matrix of the C ABI: e4m3 codes and UE8M0 scales per 128 x 128 block."""
+
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
 class MoeError(RuntimeError):
@@ -65,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.moe_route.argtypes = [CFG, I64, P, P, P, P, P, P, SZ, P]
         L.moe_dispatch.argtypes = [CFG, I64, P, P, P, P, P, SZ, P]
         L.moe_forward.argtypes = [CFG, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        FP8P = ctypes.POINTER(Fp8Matrix)
+        L.moe_forward_fp8.argtypes = [CFG, I64, P, P, P, FP8P, FP8P, FP8P, FP8P, FP8P, FP8P, P, P, P, P, SZ, P]
         L.moe_forward_host.argtypes = [CFG, I64, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.moe_workspace_release.argtypes = [P]
         L.moe_device_status.argtypes = [CFG, I64, P, SZ, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32), P]
@@ -181,6 +190,25 @@ def forward(cfg, T, x, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y, ws, topk_idx_out=No
                                             _ptr(W3), _ptr(W2), _ptr(Ws1), _ptr(Ws3), _ptr(Ws2), _ptr(y),
                                             _ptr(topk_idx_out), _ptr(gates_out), _ptr(ws), ws_bytes,
                                             _stream(stream)))
+
+
+def _fp8(m):
+    """(codes, scales) tensors -> a moe_fp8_matrix pointer (None stays NULL)."""
+    if m is None:
+        return None
+    codes, scales = m
+    return ctypes.pointer(Fp8Matrix(_ptr(codes), _ptr(scales)))
+
+
+def forward_fp8(cfg, T, x, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y, ws, topk_idx_out=None, gates_out=None,
+                ws_bytes=None, stream=None):
+    """moe_forward with FP8 expert weights; each of W1 .. Ws2 is a (codes, scales)
+    pair of uint8 tensors (e4m3 codes [rows, cols], UE8M0 scales [rows/128, cols/128])."""
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    _check("moe_forward_fp8", lib().moe_forward_fp8(ctypes.byref(cfg), T, _ptr(x), _ptr(W_r), _ptr(b), _fp8(W1),
+                                                    _fp8(W3), _fp8(W2), _fp8(Ws1), _fp8(Ws3), _fp8(Ws2), _ptr(y),
+                                                    _ptr(topk_idx_out), _ptr(gates_out), _ptr(ws), ws_bytes,
+                                                    _stream(stream)))
 
 
 def forward_host(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, ws_bytes=None,

@@ -73,24 +73,58 @@ constexpr int kTokMaps = 3;                       // token boxes of 32, 64 and 1
 constexpr int kHalfBytes = 128 * kBK * 2;         // 16 KB: 128 weight rows of one half
 constexpr int kATileBytes = 2 * kHalfBytes;       // 32 KB: this CTA's rows of both halves
 constexpr int kMaxStageBytes = kATileBytes + (kMaxTok / 2 / kTokBox) * kBoxBytes;  // 48 KB
-constexpr int kRingBytes = 52 * 4096;             // 208 KB of variable-size stages
 constexpr int kBufCols = 256;                     // fp32 columns per accumulator buffer
 constexpr int kTmemCols = 2 * kBufCols;           // 2 buffers
 constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kCvtWarps = 4;                      // FP8 weights: dequantising warps
 constexpr int kRing = 8;                          // unit ids in flight between the roles
 constexpr int kTileBytes = 32 * 32 * 2;           // a warp's dense 32 x 32 bf16 tile (TMA store box)
 constexpr int kTBytes = kEpiWarps * kTileBytes;        // one tile per epilogue warp
-constexpr int kBarrierBytes = 512;
-constexpr int kSmemBytes = kRingBytes + kTBytes + 1024 + kBarrierBytes;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kMaxStageBytes * 3 <= kRingBytes, "ring holds three full stages");
+constexpr int kA8Bytes = 2 * 128 * kBK;           // 16 KB: the fp8 codes of a CTA's 256 weight rows x 64 K
+constexpr int kFp8Block = 128;                    // FP8 scale block (rows and columns)
+
+// Shared-memory plan. bf16 weights: one ring of variable-size stages (this
+// CTA's 256 weight rows x 64 K in bf16, then the token box). FP8 weights: the
+// ring holds the fp8 codes (16 KB) and the token box; the converter warps
+// write the dequantised bf16 weight tile of each stage into one of kConv
+// slots, which the MMAs read with the stage's token box.
+template <bool FP8>
+struct Plan;
+template <>
+struct Plan<false> {
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kRingBytes = 52 * 4096;   // 208 KB
+  static constexpr int kABytes = kATileBytes;    // weight bytes at the head of a stage
+  static constexpr int kConv = 1;                // (no conversion slots; 1 keeps the arithmetic defined)
+  static constexpr int kConvBytes = 0;
+  static constexpr int kBarrierBytes = 512;
+};
+template <>
+struct Plan<true> {
+  static constexpr int kThreads = 64 + 32 * (kEpiWarps + kCvtWarps);
+  static constexpr int kRingBytes = 36 * 4096;   // 144 KB
+  static constexpr int kABytes = kA8Bytes;
+  static constexpr int kConv = 2;
+  static constexpr int kConvBytes = kConv * kATileBytes;
+  static constexpr int kBarrierBytes = 1024;
+};
+template <bool FP8>
+constexpr int smem_bytes() {
+  return Plan<FP8>::kRingBytes + Plan<FP8>::kConvBytes + kTBytes + 1024 + Plan<FP8>::kBarrierBytes;
+}
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory budget");
+static_assert(kMaxStageBytes * 3 <= Plan<false>::kRingBytes, "ring holds three full stages");
+static_assert((kA8Bytes + (kMaxTok / 2 / kTokBox) * kBoxBytes) * 4 <= Plan<true>::kRingBytes,
+              "FP8 ring holds four full stages");
 static_assert(kEpiWarps % 4 == 0, "whole quadrants");
 static_assert(kMaxTok <= kBufCols && kMaxTok % (2 * kTokBox) == 0, "token chunk");
 
 enum Mode : int { kSwiGLU = 0, kGateDown = 1 };
 
 struct TcParams {
+  // bf16 weights: bf16 maps of 64 x 128 boxes (128-byte swizzle; the down
+  // GEMM's A maps have 256-row boxes). FP8 weights: uint8 maps of the e4m3
+  // codes, 64-byte x 128-row boxes (256 rows for the down GEMM), unswizzled.
   CUtensorMap a0_routed;  // W1 [N*F, d]      | W2 [N*d, F]
   CUtensorMap a1_routed;  // W3 [N*F, d]      | unused
   CUtensorMap a0_shared;  // Ws1 [nsF, d]     | Ws2 [d, nsF]
@@ -115,6 +149,13 @@ struct TcParams {
   int out_row0_shared;           // first row of the shared MLP's rows in o_shared (0 | R)
   const float* gate_perm;        // [R] (gate-down mode)
   unsigned* status;
+  // FP8 weights: UE8M0 block scales [rows / 128, K / 128] of a0 / a1 (routed,
+  // shared), and the number of 128-row blocks of each (for clamping)
+  const uint8_t* s0_routed;
+  const uint8_t* s1_routed;
+  const uint8_t* s0_shared;
+  const uint8_t* s1_shared;
+  int sblocks_routed, sblocks_shared;
 };
 
 struct Unit {
@@ -186,10 +227,74 @@ struct Shared {
   int abort_flag;
   uint32_t consumed;           // stage fills the MMA issuer observed complete
 };
-static_assert(sizeof(Shared) <= kBarrierBytes, "barrier block");
+static_assert(sizeof(Shared) <= 512, "barrier block");
+
+// The FP8 path's extra state (after Shared, inside the barrier block).
+struct SharedFp8 {
+  uint64_t conv_full[2];       // CTA 0: both CTAs' converters wrote the slot
+  uint64_t conv_empty[2];      // both: the pair MMAs finished reading the slot
+  int cvt_unit[2];             // the converter leader's unit for the converter warps
+  int cvt_info[2][3];          // its (g, f, tok0)
+  int cvt_ok;                  // the leader's waits for the current stage succeeded
+  uint32_t seen;               // stage fills this CTA's converters observed complete
+};
+static_assert(512 + sizeof(SharedFp8) <= Plan<true>::kBarrierBytes, "FP8 barrier block");
 
 // Barrier among the epilogue warps only (id 1; id 0 is __syncthreads).
 MOE_DEV void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
+// Barrier among the FP8 converter warps only (id 2).
+MOE_DEV void cvt_sync() { asm volatile("bar.sync 2, %0;" ::"n"(32 * kCvtWarps) : "memory"); }
+
+// f16 pair -> the bf16 pair of its values times 2^-112, for f16 values
+// converted from e4m3: they carry 3 mantissa bits and are never f16
+// subnormals, so moving the f16 exponent field (5 bits) into the low bits of
+// the bf16 one and keeping the top 7 mantissa bits is exact and leaves each
+// value scaled by 2^(15 - 127). Zero stays zero.
+MOE_DEV uint32_t f16x2_to_bf16x2_scaled(uint32_t h) { return ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u); }
+
+// Four e4m3 codes (lowest byte first) -> two bf16 pairs (the values times
+// 2^-112); cvt.f16x2.e4m3x2 is exact.
+MOE_DEV void e4m3x4_to_bf16x4_scaled(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  uint32_t a, b;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(a), "=r"(b)
+      : "r"(w));
+  lo = f16x2_to_bf16x2_scaled(a);
+  hi = f16x2_to_bf16x2_scaled(b);
+}
+
+MOE_DEV uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// bf16 pair (f, f) with f = 2^e, -126 <= e <= 127.
+MOE_DEV uint32_t bf16x2_pow2(int e) {
+  const uint32_t b = (uint32_t)(e + 127) << 7;
+  return b | (b << 16);
+}
+
+// 16 e4m3 codes -> 16 bf16 values, each code value times 2^(sb - 127):
+// multiplied by 2^(112 + sb - 127) in one or (for sb > 142) two exact steps.
+MOE_DEV void dequant16(const uint4 w, int sb, uint32_t (&o)[8]) {
+  const int e = sb - 15;                    // exponent of the total factor
+  const int e1 = e > 127 ? 127 : e;
+  const uint32_t f1 = bf16x2_pow2(e1);
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t lo, hi;
+    e4m3x4_to_bf16x4_scaled(words[i], lo, hi);
+    o[2 * i] = mul_bf16x2(lo, f1);
+    o[2 * i + 1] = mul_bf16x2(hi, f1);
+  }
+  if (e > 127) {
+    const uint32_t f2 = bf16x2_pow2(e - 127);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = mul_bf16x2(o[i], f2);
+  }
+}
 
 MOE_DEV int load_volatile(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
 
@@ -208,21 +313,29 @@ MOE_DEV void store_row32(__nv_bfloat16* dst, int ncols, const uint4 (&v)[4]) {
   }
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
+template <int MODE, bool FP8>
+__global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
+  using PL = Plan<FP8>;
+  constexpr int kRingBytes = PL::kRingBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* tiles = reinterpret_cast<float*>(smem + kRingBytes);
-  Shared& sh = *reinterpret_cast<Shared*>(smem + kRingBytes + kTBytes);
+  uint8_t* conv = smem + kRingBytes;  // FP8: the dequantised weight slots
+  float* tiles = reinterpret_cast<float*>(conv + PL::kConvBytes);
+  Shared& sh = *reinterpret_cast<Shared*>(reinterpret_cast<uint8_t*>(tiles) + kTBytes);
+  SharedFp8& shf = *reinterpret_cast<SharedFp8*>(reinterpret_cast<uint8_t*>(&sh) + 512);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: issues the pair MMAs and takes the units
   const bool first = rank == 0;
   const int total_units = __ldg(p.unit_base + p.N + 1);
-  // this CTA's rows of each 256-row weight half, and the offset between halves
-  const int rank_rows = 128 * (int)rank;
-  const int half_rows = MODE == kSwiGLU ? 0 : 256;
+  // Weight rows of this CTA. SwiGLU: rows 128 r .. 128 r + 127 of the unit's
+  // 256 features, taken from W1 (half 0) and from W3 (half 1). Down GEMM:
+  // rows 256 r .. 256 r + 255 of the unit's 512 output columns, one
+  // contiguous 256-row box whose first and second 128 rows are halves 0 and
+  // 1; so TMEM lane l of half h in CTA r is output column 256 r + 128 h + l.
+  const int rank_rows = (MODE == kSwiGLU ? 128 : 256) * (int)rank;
+  const int half_cols = MODE == kSwiGLU ? 0 : 128;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
@@ -235,11 +348,19 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
     }
     for (int q = 0; q < kRing; ++q) {
       mbar_init(&sh.ring_full[q], 1);
-      mbar_init(&sh.ring_empty[q], 4);  // both CTAs: producer or MMA issuer, epilogue leader
+      // both CTAs: producer or MMA issuer, epilogue leader (and FP8 converter leader)
+      mbar_init(&sh.ring_empty[q], FP8 ? 6 : 4);
     }
     mbar_init(&sh.drained, 1);
     sh.abort_flag = 0;
     sh.consumed = 0;
+    if (FP8) {
+      for (int c = 0; c < PL::kConv; ++c) {
+        mbar_init(&shf.conv_full[c], 2);
+        mbar_init(&shf.conv_empty[c], 1);
+      }
+      shf.seen = 0;
+    }
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -345,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         // single box beats several small ones even with rows to spare)
         const int tmap = half_n <= kTokBox ? 0 : (half_n <= 2 * kTokBox ? 1 : 2);
         const int nbox = 1 << tmap;  // in 32-row granules
-        const uint32_t tx = kATileBytes + nbox * kBoxBytes;
+        const uint32_t tx = PL::kABytes + nbox * kBoxBytes;
         const int rowA = (shared ? 0 : un.g * p.a_rows_per_expert) + un.f * p.tile_cols + rank_rows;
         const int rowB = __ldg(p.grp_row0 + un.g) + un.tok0 + (int)rank * half_n;
         const CUtensorMap* ta0 = shared ? &p.a0_shared : &p.a0_routed;
@@ -363,12 +484,21 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           head = pos + tx;
           sh.slot_off[s] = pos;
           uint8_t* a_dst = smem + pos;
-          uint8_t* b_dst = a_dst + kATileBytes;
-          const uint32_t full_bar = in_first(&sh.full[s]);
-          if (first) mbar_arrive_expect_tx(&sh.full[s], 2 * tx);  // this CTA's bytes and the peer's
-          tma_load_2d_pair(a_dst, ta0, full_bar, kc * kBK, rowA, pol);
-          tma_load_2d_pair(a_dst + kHalfBytes, ta1, full_bar, kc * kBK, rowA + half_rows, pol);
-          tma_load_2d_pair(b_dst, tb, full_bar, kc * kBK, rowB, pol_shared);
+          uint8_t* b_dst = a_dst + PL::kABytes;
+          if (FP8) {
+            // every CTA's bytes complete on its own stage barrier, which its
+            // converter warps wait on; the codes are 64 bytes per row
+            mbar_arrive_expect_tx(&sh.full[s], tx);
+            tma_load_2d_hint(a_dst, ta0, &sh.full[s], kc * kBK, rowA, pol);
+            if (MODE == kSwiGLU) tma_load_2d_hint(a_dst + kA8Bytes / 2, ta1, &sh.full[s], kc * kBK, rowA, pol);
+            tma_load_2d_hint(b_dst, tb, &sh.full[s], kc * kBK, rowB, pol_shared);
+          } else {
+            const uint32_t full_bar = in_first(&sh.full[s]);
+            if (first) mbar_arrive_expect_tx(&sh.full[s], 2 * tx);  // this CTA's bytes and the peer's
+            tma_load_2d_pair(a_dst, ta0, full_bar, kc * kBK, rowA, pol);  // SwiGLU: 128 W1 rows; down: 256 rows
+            if (MODE == kSwiGLU) tma_load_2d_pair(a_dst + kHalfBytes, ta1, full_bar, kc * kBK, rowA, pol);
+            tma_load_2d_pair(b_dst, tb, full_bar, kc * kBK, rowB, pol_shared);
+          }
         }
         if (!ok) break;
       }
@@ -411,14 +541,20 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
         const uint32_t d0 = tmem_base + base, d1 = tmem_base + base + stride;
         for (int kc = 0; kc < nk; ++kc) {
           const uint32_t s = consumed % kSlots, ph = (consumed / kSlots) & 1u;
-          if (!mbar_wait_cluster_bounded(&sh.full[s], ph, abort_flag)) {
+          // FP8: the converted slot of this fill (both CTAs' converters have
+          // observed its bytes land before they released it)
+          const uint32_t c = FP8 ? consumed % PL::kConv : 0u;
+          const bool landed = FP8 ? mbar_wait_cluster_bounded(&shf.conv_full[c], (consumed / PL::kConv) & 1u, abort_flag)
+                                  : mbar_wait_cluster_bounded(&sh.full[s], ph, abort_flag);
+          if (!landed) {
             ok = false;
             break;
           }
           ++consumed;
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + *reinterpret_cast<volatile uint32_t*>(&sh.slot_off[s]));
-          const uint32_t b_addr = a_addr + kATileBytes;
+          const uint32_t stage_addr = smem_u32(smem + *reinterpret_cast<volatile uint32_t*>(&sh.slot_off[s]));
+          const uint32_t a_addr = FP8 ? smem_u32(conv + c * kATileBytes) : stage_addr;
+          const uint32_t b_addr = stage_addr + PL::kABytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32);
@@ -427,6 +563,10 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           }
           umma_commit_pair(smem_u32(&sh.empty[s]));
           umma_commit_pair(peer(&sh.empty[s]));
+          if (FP8) {
+            umma_commit_pair(smem_u32(&shf.conv_empty[c]));
+            umma_commit_pair(peer(&shf.conv_empty[c]));
+          }
         }
         if (ok) {
           for (int b = 0; b < 2; ++b)
@@ -450,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
       if (!mbar_wait_cluster_bounded(&sh.drained, 0, &no_abort)) set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------ epilogue --
     const int q = warp & 3;                  // TMEM lane quadrant this warp may access
     const int ew = warp - 2;                 // epilogue warp: its transpose tile
@@ -514,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
 #pragma unroll 1
       for (int hh = 0; hh < kHalves; ++hh) {
         // this warp's 32 output columns of the unit
-        const int c0 = un.f * p.tile_cols + half_rows * hh + rank_rows + 32 * q;
+        const int c0 = un.f * p.tile_cols + rank_rows + half_cols * hh + 32 * q;
 #pragma unroll 1
         for (int j0 = 32 * sub; j0 < un.ntok; j0 += 32 * (kEpiWarps / 4)) {
           const int tok = j0 + lane;
@@ -607,14 +747,116 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_tc_kernel(const __gri
           }
       }
     }
+  } else if (FP8) {
+    // ----------------------------------------- FP8 converters (kCvtWarps) --
+    // Per fill, in the producer's order: wait for this CTA's bytes and for a
+    // free conversion slot, write the 256 x 64 dequantised bf16 weights in the
+    // 128-byte-swizzled layout the MMA descriptors expect (the layout a bf16
+    // TMA load would have produced), then tell the MMA issuer. A leader does
+    // the waits and the other warps follow its decision.
+    const int ct = threadIdx.x - 32 * (2 + kEpiWarps);  // 0 .. 32 kCvtWarps - 1
+    const bool cleader = ct == 0;
+    uint32_t j = 0;  // fills converted
+    bool alive = true;
+    for (int i = 0; alive; ++i) {
+      if (cleader) {
+        int u = -2;
+        const int qr = i % kRing;
+        if (mbar_wait_cluster_bounded(&sh.ring_full[qr], (i / kRing) & 1, abort_flag)) {
+          u = load_volatile(&sh.ring[qr]);
+          if (first) mbar_arrive(&sh.ring_empty[qr]);
+          else mbar_arrive_cluster(in_first(&sh.ring_empty[qr]));
+          if (u >= 0) {
+            const Unit un = decode_unit(p, u);
+            shf.cvt_info[i & 1][0] = un.g;
+            shf.cvt_info[i & 1][1] = un.f;
+          }
+        }
+        if (u == -2) {
+          *abort_flag = 1;
+          set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
+        }
+        shf.cvt_unit[i & 1] = u;
+      }
+      cvt_sync();
+      if (load_volatile(&shf.cvt_unit[i & 1]) < 0) break;
+      const int g = load_volatile(&shf.cvt_info[i & 1][0]);
+      const int f = load_volatile(&shf.cvt_info[i & 1][1]);
+      const bool shared = g == p.N;
+      const int K = shared ? p.k_shared : p.k_routed;
+      const int nk = K / kBK;                 // K is a multiple of 128 on this path
+      const int nkb = K / kFp8Block;          // <= 64
+      const int rowA = (shared ? 0 : g * p.a_rows_per_expert) + f * p.tile_cols + rank_rows;
+      const int sblocks = shared ? p.sblocks_shared : p.sblocks_routed;
+      // this CTA's two 128-row halves: SwiGLU W1 / W3 rows of the same block,
+      // down GEMM two consecutive W2 blocks (a block past the matrix, whose
+      // rows load as zeros, takes the last block's scales)
+      const int rb0 = min(rowA / kFp8Block, sblocks - 1);
+      const int rb1 = MODE == kSwiGLU ? rb0 : min(rowA / kFp8Block + 1, sblocks - 1);
+      const uint8_t* sc0 = (shared ? p.s0_shared : p.s0_routed) + (int64_t)rb0 * nkb;
+      const uint8_t* sc1 = (MODE == kSwiGLU ? (shared ? p.s1_shared : p.s1_routed) : (shared ? p.s0_shared : p.s0_routed)) +
+                           (int64_t)rb1 * nkb;
+      // lane l holds the scale bytes of K blocks l and l + 32 of both halves
+      const int l = ct & 31;
+      const int sA0 = l < nkb ? __ldg(sc0 + l) : 0, sA1 = l + 32 < nkb ? __ldg(sc0 + l + 32) : 0;
+      const int sB0 = l < nkb ? __ldg(sc1 + l) : 0, sB1 = l + 32 < nkb ? __ldg(sc1 + l + 32) : 0;
+      for (int kc = 0; kc < nk; ++kc, ++j) {
+        const uint32_t s = j % kSlots, c = j % PL::kConv;
+        if (cleader) {
+          const bool ok = mbar_wait_bounded(&sh.full[s], (j / kSlots) & 1u, abort_flag) &&
+                          mbar_wait_cluster_bounded(&shf.conv_empty[c], ((j / PL::kConv) & 1u) ^ 1u, abort_flag);
+          if (ok) shf.seen = j + 1;
+          else {
+            *abort_flag = 1;
+            set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
+          }
+          shf.cvt_ok = ok;
+        }
+        cvt_sync();
+        if (!load_volatile(&shf.cvt_ok)) {
+          alive = false;
+          break;
+        }
+        const int kb = kc >> 1;  // 64-wide K block -> 128-wide scale block
+        const int sb0 = __shfl_sync(0xffffffffu, kb < 32 ? sA0 : sA1, kb & 31);
+        const int sb1 = __shfl_sync(0xffffffffu, kb < 32 ? sB0 : sB1, kb & 31);
+        const uint32_t raw = smem_u32(smem) + *reinterpret_cast<volatile uint32_t*>(&sh.slot_off[s]);
+        const uint32_t dst = smem_u32(conv) + c * kATileBytes;
+        constexpr int kPieces = kA8Bytes / 16 / (32 * kCvtWarps);  // 16-byte pieces per thread
+        uint4 wv[kPieces];  // all loads first: independent work for the conversion below
+#pragma unroll
+        for (int it = 0; it < kPieces; ++it) {
+          const int v = ct + 32 * kCvtWarps * it;  // 16-byte piece: row v / 4 (of 256), bytes 16 (v % 4) ..
+          wv[it] = ld_shared_v4(raw + (v >> 2) * kBK + (v & 3) * 16);
+        }
+#pragma unroll
+        for (int it = 0; it < kPieces; ++it) {
+          const int v = ct + 32 * kCvtWarps * it;
+          const int r = v >> 2, q4 = v & 3;
+          uint32_t o[8];
+          dequant16(wv[it], r < 128 ? sb0 : sb1, o);
+          const int rr = r & 127;
+          const uint32_t row = dst + (r >> 7) * kHalfBytes + rr * (kBK * 2);
+          st_shared_v4(row + (((2 * q4) ^ (rr & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+          st_shared_v4(row + (((2 * q4 + 1) ^ (rr & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+        }
+        fence_proxy_async_smem();  // the tensor cores read the slot through the async proxy
+        cvt_sync();
+        if (cleader) {
+          if (first) mbar_arrive(&shf.conv_full[c]);
+          else mbar_arrive_cluster(in_first(&shf.conv_full[c]));
+        }
+      }
+    }
   }
 
-  if (warp >= 2 && lane == 0) bulk_wait_group_all();  // epilogue stores complete
+  if (warp >= 2 && warp < 2 + kEpiWarps && lane == 0) bulk_wait_group_all();  // epilogue stores complete
   __syncthreads();
-  if (warp == 0 && lane == 0 && first) {
+  if (warp == 0 && lane == 0 && (first || FP8)) {
     // wait for any stage fill that was issued but never observed complete
-    // (its bytes from both CTAs land on this CTA's stage barrier)
-    for (uint32_t j = sh.consumed; j < fills; ++j) {
+    // (bf16: the bytes of both CTAs land on the first CTA's stage barrier;
+    // FP8: every CTA's land on its own and its converters observe them)
+    for (uint32_t j = FP8 ? shf.seen : sh.consumed; j < fills; ++j) {
       const uint32_t s = j % kSlots, ph = (j / kSlots) & 1u;
       int dummy = 0;
       if (!mbar_wait_cluster_bounded(&sh.full[s], ph, &dummy)) {
@@ -648,7 +890,12 @@ bool make_store_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
   return make_tmap_bf16_swz(m, base, rows, cols, 32, 32, 64);
 }
 
-template <int MODE>
+// FP8 weight codes: 64 bytes x box_rows rows, unswizzled (the converters read them row by row).
+bool make_tmap_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  return make_tmap_u8(m, base, rows, cols, kBK, box_rows);
+}
+
+template <int MODE, bool FP8>
 cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s, bool programmatic) {
   // per device: the shared-memory opt-in done and the resident cluster count
   static std::mutex mu;
@@ -665,8 +912,8 @@ cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s, bool 
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.blockDim = dim3(Plan<FP8>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes<FP8>();
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -674,12 +921,12 @@ cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s, bool 
   {
     std::lock_guard<std::mutex> lock(mu);
     if (max_clusters_of[dev] == 0) {
-      cudaError_t e = cudaFuncSetAttribute(expert_gemm_tc_kernel<MODE>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      cudaError_t e = cudaFuncSetAttribute(expert_gemm_tc_kernel<MODE, FP8>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<FP8>());
       if (e != cudaSuccess) return e;
       cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
       int n = 0;
-      e = cudaOccupancyMaxActiveClusters(&n, expert_gemm_tc_kernel<MODE>, &cfg);
+      e = cudaOccupancyMaxActiveClusters(&n, expert_gemm_tc_kernel<MODE, FP8>, &cfg);
       if (e != cudaSuccess) return e;
       max_clusters_of[dev] = n > 0 ? n : 1;
     }
@@ -688,7 +935,7 @@ cudaError_t launch_one(const TcParams& prm, int max_units, cudaStream_t s, bool 
   if (max_units < clusters) clusters = max_units > 0 ? max_units : 1;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.numAttrs = programmatic ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, expert_gemm_tc_kernel<MODE>, prm);
+  return cudaLaunchKernelEx(&cfg, expert_gemm_tc_kernel<MODE, FP8>, prm);
 }
 
 }  // namespace
@@ -701,11 +948,16 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   const int64_t chunks_bound =
       (p.R + kMaxTok - 1) / kMaxTok + p.N + (p.ns > 0 ? (p.T + kMaxTok - 1) / kMaxTok : 0);
 
+  const bool fp8 = a.fp8;
+  // weight maps: bf16 tiles, or the FP8 codes (plus their block scales)
+  auto wmap = [&](CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    return fp8 ? make_tmap_codes(m, base, rows, cols, box_rows) : make_tmap(m, base, rows, cols, box_rows);
+  };
   TcParams g1{};
-  bool ok = make_tmap(&g1.a0_routed, a.W1, (uint64_t)p.N * p.F, p.d, 128) &&
-            make_tmap(&g1.a1_routed, a.W3, (uint64_t)p.N * p.F, p.d, 128) &&
-            make_tmap(&g1.a0_shared, a.Ws1, (uint64_t)p.nsF, p.d, 128) &&
-            make_tmap(&g1.a1_shared, a.Ws3, (uint64_t)p.nsF, p.d, 128) &&
+  bool ok = wmap(&g1.a0_routed, a.W1, (uint64_t)p.N * p.F, p.d, 128) &&
+            wmap(&g1.a1_routed, a.W3, (uint64_t)p.N * p.F, p.d, 128) &&
+            wmap(&g1.a0_shared, a.Ws1, (uint64_t)p.nsF, p.d, 128) &&
+            wmap(&g1.a1_shared, a.Ws3, (uint64_t)p.nsF, p.d, 128) &&
             make_token_tmaps(g1.b_routed, a.x_perm, (uint64_t)p.R, p.d) &&
             make_token_tmaps(g1.b_shared, p.ns ? a.x : nullptr, (uint64_t)p.T, p.d) &&
             make_store_tmap(&g1.o_routed, a.h_perm, (uint64_t)p.R, p.F) &&
@@ -729,15 +981,22 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g1.ld_shared = p.nsF;
   g1.gate_perm = nullptr;
   g1.status = a.status;
+  g1.s0_routed = a.W1s;
+  g1.s1_routed = a.W3s;
+  g1.s0_shared = a.Ws1s;
+  g1.s1_shared = a.Ws3s;
+  g1.sblocks_routed = (int)((int64_t)p.N * p.F / kFp8Block);
+  g1.sblocks_shared = p.nsF / kFp8Block;
   const int64_t max_cols1 = p.F > p.nsF ? p.F : p.nsF;
   const int64_t units1 = chunks_bound * ((max_cols1 + kTcBN1 - 1) / kTcBN1);
-  cudaError_t err = launch_one<kSwiGLU>(g1, (int)(units1 < sms ? units1 : sms), s, false);
+  const int grid1 = (int)(units1 < sms ? units1 : sms);
+  cudaError_t err = fp8 ? launch_one<kSwiGLU, true>(g1, grid1, s, false) : launch_one<kSwiGLU, false>(g1, grid1, s, false);
   if (err == cudaSuccess && between) err = cudaEventRecord(between, s);
   if (err != cudaSuccess) return err;
 
   TcParams g2{};
-  ok = make_tmap(&g2.a0_routed, a.W2, (uint64_t)p.N * p.d, p.F, 128) &&
-       make_tmap(&g2.a0_shared, a.Ws2, (uint64_t)p.d, p.nsF, 128) &&
+  ok = wmap(&g2.a0_routed, a.W2, (uint64_t)p.N * p.d, p.F, 256) &&
+       wmap(&g2.a0_shared, a.Ws2, (uint64_t)p.d, p.nsF, 256) &&
        make_token_tmaps(g2.b_routed, a.h_perm, (uint64_t)p.R, p.F) &&
        make_token_tmaps(g2.b_shared, p.ns ? a.h_sh : nullptr, (uint64_t)p.T, p.nsF) &&
        make_store_tmap(&g2.o_routed, a.y_rows, (uint64_t)(p.R + p.T), p.d) &&
@@ -761,10 +1020,15 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g2.ld_shared = p.d;
   g2.gate_perm = a.gate_perm;
   g2.status = a.status;
+  g2.s0_routed = a.W2s;
+  g2.s0_shared = a.Ws2s;
+  g2.sblocks_routed = (int)((int64_t)p.N * p.d / kFp8Block);
+  g2.sblocks_shared = p.d / kFp8Block;
   const int64_t units2 = chunks_bound * ((p.d + kTcBN2 - 1) / kTcBN2);
+  const int grid2 = (int)(units2 < sms ? units2 : sms);
   // the down GEMM overlaps the SwiGLU GEMM's drain unless an event must be
   // recorded between the two
-  return launch_one<kGateDown>(g2, (int)(units2 < sms ? units2 : sms), s, !between);
+  return fp8 ? launch_one<kGateDown, true>(g2, grid2, s, !between) : launch_one<kGateDown, false>(g2, grid2, s, !between);
 }
 
 }  // namespace moe

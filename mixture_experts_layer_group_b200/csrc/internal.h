@@ -71,6 +71,10 @@ struct DispatchBuffers {
 // base or an empty matrix gives a zeroed map that must not be used.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                     uint32_t box_rows, bool swizzle128);
+// uint8 row-major [rows, cols] (FP8 codes) with a box of box_cols bytes x
+// box_rows rows, no swizzle, 256-byte L2 promotion; zero fill outside.
+bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                  uint32_t box_rows);
 // The same with a swizzle of 0, 64 or 128 bytes.
 bool make_tmap_bf16_swz(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                         uint32_t box_rows, int swizzle_bytes);
@@ -117,6 +121,15 @@ struct GemmArgs {
   const float* gate_perm;
   unsigned* status;
   int* sched;           // [2] unit counters of the two tensor-core launches
+  // FP8 expert weights: W1 .. Ws2 above hold the e4m3 codes (uint8, same
+  // shapes) and these their UE8M0 scales, one byte per 128 x 128 block
+  bool fp8 = false;
+  const uint8_t* W1s = nullptr;
+  const uint8_t* W3s = nullptr;
+  const uint8_t* W2s = nullptr;
+  const uint8_t* Ws1s = nullptr;
+  const uint8_t* Ws3s = nullptr;
+  const uint8_t* Ws2s = nullptr;
 };
 
 // Tensor-core (bf16) expert GEMMs: SwiGLU projection then gated down

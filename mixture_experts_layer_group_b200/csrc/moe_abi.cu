@@ -166,10 +166,16 @@ DispatchBuffers dispatch_buffers(const Layout& L, void* ws, const int32_t* idx, 
   return db;
 }
 
+// Scale pointers of FP8 expert weights (W1, W3, W2, Ws1, Ws3, Ws2), or null for bf16 / fp32 weights.
+struct Fp8Scales {
+  const uint8_t* s[6];
+};
+
 moe_status forward_device(const Problem& p, const Layout& L, const void* x, const void* W_r,
                           const float* b, const void* W1, const void* W3, const void* W2,
                           const void* Ws1, const void* Ws3, const void* Ws2, void* y,
-                          int32_t* idx_out, float* gates_out, void* ws, cudaStream_t s) {
+                          int32_t* idx_out, float* gates_out, void* ws, cudaStream_t s,
+                          const Fp8Scales* fp8 = nullptr) {
   int32_t* idx = at<int32_t>(ws, L.idx);
   float* gates = at<float>(ws, L.gates);
   cudaError_t e0 = cudaMemsetAsync(at<void>(ws, L.status), 0, 4, s);
@@ -206,6 +212,15 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
   ga.gate_perm = db.gate_perm;
   ga.status = db.status;
   ga.sched = at<int>(ws, L.sched);
+  if (fp8) {
+    ga.fp8 = true;
+    ga.W1s = fp8->s[0];
+    ga.W3s = fp8->s[1];
+    ga.W2s = fp8->s[2];
+    ga.Ws1s = p.ns ? fp8->s[3] : nullptr;
+    ga.Ws3s = p.ns ? fp8->s[4] : nullptr;
+    ga.Ws2s = p.ns ? fp8->s[5] : nullptr;
+  }
   e = tc ? launch_expert_gemms_tc(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr)
          : launch_expert_gemms_simt(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr);
   if (e == cudaSuccess) e = mark_stage(5, s);
@@ -389,6 +404,39 @@ moe_status moe_forward(const moe_cfg* cfg, int64_t T, const void* x, const void*
   if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
   st = forward_device(p, L, x, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y, topk_idx_out, gates_out, ws,
                       (cudaStream_t)stream);
+  if (st != MOE_OK) return st;
+  cudaError_t e = note_device_use(ws, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status moe_forward_fp8(const moe_cfg* cfg, int64_t T, const void* x, const void* W_r, const float* b,
+                           const moe_fp8_matrix* W1, const moe_fp8_matrix* W3, const moe_fp8_matrix* W2,
+                           const moe_fp8_matrix* Ws1, const moe_fp8_matrix* Ws3, const moe_fp8_matrix* Ws2,
+                           void* y, int32_t* topk_idx_out, float* gates_out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
+  if (st != MOE_OK) return st;
+  if (p.dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  constexpr int kBlock = 128, kMaxK = 8192;  // block size; K / 128 scale blocks per lane pair
+  if (p.d % kBlock || p.F % kBlock || p.nsF % kBlock || p.d > kMaxK || p.F > kMaxK || p.nsF > kMaxK)
+    return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!x || !y || !aligned16(x) || !aligned16(y) || !W_r || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
+  if (b && (reinterpret_cast<uintptr_t>(b) & 3u)) return MOE_ERR_INVALID_ARG;
+  const moe_fp8_matrix* m[6] = {W1, W3, W2, Ws1, Ws3, Ws2};
+  for (int i = 0; i < 6; ++i) {
+    const bool need = i < 3 || p.ns > 0;
+    if (!need) continue;
+    if (!m[i] || !m[i]->codes || !m[i]->scales || !aligned16(m[i]->codes)) return MOE_ERR_INVALID_ARG;
+  }
+  Layout L = make_layout(p);
+  if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
+  Fp8Scales sc{};
+  for (int i = 0; i < 6; ++i) sc.s[i] = (i < 3 || p.ns > 0) ? m[i]->scales : nullptr;
+  auto codes = [&](int i) -> const void* { return (i < 3 || p.ns > 0) ? m[i]->codes : nullptr; };
+  st = forward_device(p, L, x, W_r, b, codes(0), codes(1), codes(2), codes(3), codes(4), codes(5), y, topk_idx_out,
+                      gates_out, ws, (cudaStream_t)stream, &sc);
   if (st != MOE_OK) return st;
   cudaError_t e = note_device_use(ws, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);

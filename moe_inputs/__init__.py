@@ -18,6 +18,14 @@ Recipe (the shapes and distributions of the five layer configurations):
   Ws2 ~ approx. N(0, 1/(n_s*d_ff))           [d, n_s*d_ff]
   "approx. N" is the Irwin-Hall sum of four uniforms rescaled to the stated
   standard deviation (same mean and variance, support +-3.46 sd).
+  FP8 expert weights (wdtype "fp8"): each expert matrix, viewed as
+  [rows, cols], is stored as e4m3 codes with one power-of-two scale per
+  128 x 128 block: block b gets the exponent e_b = e0 + (hash & 3), e0 the
+  smallest with 2^e0 * 448 >= the largest generated |value|, and each code is
+  the e4m3 value nearest (ties to even) to v * 2^-e_b for the same
+  approximately normal v as above; the scale byte is e_b + 127 (UE8M0).
+  So the dequantised weights keep the N(0, 1/fan_in) shape while the block
+  scales differ from block to block by up to 8x.
   Skewed routing (decode shape): a seeded permutation gives each expert a
   rank r_e in 1..N; column 0 of x is set to 1 and column 0 of W_r to
   o_e = -s * ln(r_e), so the router logits carry an offset whose exponential
@@ -38,6 +46,9 @@ DEVICE_LIB = os.path.join(_HERE, "libmoe_gen_device.so")
 
 # tensor ids of the counter-based generator
 TID = {"x": 0, "W_r": 1, "b": 2, "W1": 3, "W3": 4, "W2": 5, "Ws1": 6, "Ws3": 7, "Ws2": 8, "zipf": 9}
+# tensor ids of the FP8 block exponents of each expert matrix
+TID_SCALE = {"W1": 10, "W3": 11, "W2": 12, "Ws1": 13, "Ws3": 14, "Ws2": 15}
+FP8_BLOCK = 128
 IRWIN_HALL4_SD = math.sqrt(1431655765.0)  # sd of the sum of four 16-bit uniforms
 
 
@@ -62,6 +73,7 @@ class LayerShape:
     seed: int = 0
     bias: bool = False
     zipf_s: float | None = None
+    wdtype: str = "bf16"  # expert weights: "bf16" (as dtype) or "fp8" (e4m3 + 128 x 128 block scales)
 
     def with_(self, **kw) -> "LayerShape":
         return replace(self, **kw)
@@ -101,6 +113,10 @@ SHAPES["v3_prefill_t16k_bf16"] = SHAPES["v3_prefill_bf16"].with_(name="v3_prefil
 # its highest affinities (group score = the device's best expert score).
 SHAPES["v2_device_limited_bf16"] = SHAPES["v2_layer_bf16"].with_(name="v2_device_limited_bf16", n_groups=8,
                                                                    topk_groups=3, group_score="max")
+# The V3 prefill layer with FP8 expert weights (e4m3 codes, one power-of-two
+# scale per 128 x 128 block); tokens, router and bias as in the bf16 layer.
+SHAPES["v3_prefill_fp8"] = SHAPES["v3_prefill_bf16"].with_(name="v3_prefill_fp8", wdtype="fp8")
+SHAPES["v3_decode_fp8"] = SHAPES["v3_decode_bf16"].with_(name="v3_decode_fp8", wdtype="fp8")
 ORDER = ["gshard_tiny_f32", "dsmoe_2b_bf16", "v2_layer_bf16", "v3_prefill_bf16", "v3_decode_bf16"]
 
 
@@ -137,6 +153,10 @@ def _host_lib():
                                     ctypes.c_int]
         lib.gen_hash.argtypes = [ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_uint64,
                                  ctypes.c_void_p]
+        lib.gen_fp8.argtypes = [ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_int, ctypes.c_uint64,
+                                ctypes.c_uint64, ctypes.c_uint64, ctypes.c_double, ctypes.c_void_p, ctypes.c_int]
+        lib.gen_fp8_scales.argtypes = [ctypes.c_uint32, ctypes.c_uint32, ctypes.c_int, ctypes.c_uint64,
+                                       ctypes.c_uint64, ctypes.c_void_p]
         _host = lib
     return _host
 
@@ -161,6 +181,62 @@ def host_hash(seed: int, tid: int, offset: int, n: int) -> np.ndarray:
     out = np.empty(n, dtype=np.uint64)
     _host_lib().gen_hash(seed, tid, offset, n, out.ctypes.data)
     return out
+
+
+def mat_dims(shape: LayerShape, name: str) -> tuple:
+    """2-D view [rows, cols] of an expert weight tensor (routed experts stacked along rows)."""
+    d, F, N, ns = shape.d, shape.d_ff, shape.n_routed, shape.n_shared
+    return {"W1": (N * F, d), "W3": (N * F, d), "W2": (N * d, F), "Ws1": (ns * F, d), "Ws3": (ns * F, d),
+            "Ws2": (d, ns * F)}[name]
+
+
+def fp8_e0(shape: LayerShape, name: str) -> int:
+    """Smallest block exponent: 2^e0 * 448 covers the largest value the
+    generator can produce (131070 * factor, about 3.46 standard deviations)."""
+    return int(math.ceil(math.log2(131070.0 * factor_of(shape, name) / 448.0)))
+
+
+def host_fp8(shape: LayerShape, name: str, offset: int = 0, n: int | None = None) -> np.ndarray:
+    """e4m3 codes (uint8) of elements [offset, offset + n) of an expert matrix."""
+    rows, cols = mat_dims(shape, name)
+    n = rows * cols - offset if n is None else n
+    out = np.empty(n, dtype=np.uint8)
+    _host_lib().gen_fp8(shape.seed, TID[name], TID_SCALE[name], fp8_e0(shape, name), cols, offset, n,
+                        factor_of(shape, name), out.ctypes.data, _nthreads())
+    return out
+
+
+def host_fp8_scales(shape: LayerShape, name: str, offset: int = 0, n: int | None = None) -> np.ndarray:
+    """UE8M0 scale bytes of blocks [offset, offset + n) (row-major over [rows/128, cols/128])."""
+    rows, cols = mat_dims(shape, name)
+    n = (rows // FP8_BLOCK) * (cols // FP8_BLOCK) - offset if n is None else n
+    out = np.empty(n, dtype=np.uint8)
+    _host_lib().gen_fp8_scales(shape.seed, TID_SCALE[name], fp8_e0(shape, name), offset, n, out.ctypes.data)
+    return out
+
+
+def host_expert_fp8(shape: LayerShape, e: int):
+    """((q, s) of W1_e, W3_e, W2_e): codes [F, d] / [d, F] and block scales [F/128, d/128] / [d/128, F/128]."""
+    d, F = shape.d, shape.d_ff
+    n, nb = F * d, (F // FP8_BLOCK) * (d // FP8_BLOCK)
+    out = []
+    for nm, shp in (("W1", (F, d)), ("W3", (F, d)), ("W2", (d, F))):
+        q = host_fp8(shape, nm, e * n, n).reshape(shp)
+        sc = host_fp8_scales(shape, nm, e * nb, nb).reshape(shp[0] // FP8_BLOCK, shp[1] // FP8_BLOCK)
+        out.append((q, sc))
+    return tuple(out)
+
+
+def host_shared_fp8(shape: LayerShape):
+    """((q, s) of Ws1, Ws3, Ws2), or None without a shared expert."""
+    if shape.n_shared == 0:
+        return None
+    out = []
+    for nm in ("Ws1", "Ws3", "Ws2"):
+        rows, cols = mat_dims(shape, nm)
+        out.append((host_fp8(shape, nm).reshape(rows, cols),
+                    host_fp8_scales(shape, nm).reshape(rows // FP8_BLOCK, cols // FP8_BLOCK)))
+    return tuple(out)
 
 
 def bf16_to_f32(u16: np.ndarray) -> np.ndarray:

@@ -11,7 +11,8 @@ import os
 import numpy as np
 import torch
 
-from . import (DEVICE_LIB, TID, LayerShape, dims_of, f32_to_bf16, factor_of, zipf_offsets)
+from . import (DEVICE_LIB, FP8_BLOCK, TID, TID_SCALE, LayerShape, dims_of, f32_to_bf16, factor_of, fp8_e0,
+               mat_dims, zipf_offsets)
 
 _dev = None
 
@@ -28,6 +29,11 @@ def _device_lib():
         lib.gen_uniform_device.argtypes = [ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint64,
                                            ctypes.c_uint64, ctypes.c_double, ctypes.c_double,
                                            ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+        lib.gen_fp8_device.argtypes = [ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_int,
+                                       ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_double,
+                                       ctypes.c_void_p, ctypes.c_void_p]
+        lib.gen_fp8_scales_device.argtypes = [ctypes.c_uint32, ctypes.c_uint32, ctypes.c_int, ctypes.c_uint64,
+                                              ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]
         _dev = lib
     return _dev
 
@@ -64,9 +70,30 @@ def device_tensor(shape: LayerShape, name: str, device="cuda") -> torch.Tensor:
     return out
 
 
+def device_fp8(shape: LayerShape, name: str, device="cuda"):
+    """(codes uint8 [rows, cols], scales uint8 [rows/128, cols/128]) of an FP8 expert matrix."""
+    rows, cols = mat_dims(shape, name)
+    stream = torch.cuda.current_stream(device).cuda_stream
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=device)
+    sc = torch.empty((rows // FP8_BLOCK, cols // FP8_BLOCK), dtype=torch.uint8, device=device)
+    lib = _device_lib()
+    rc = lib.gen_fp8_device(shape.seed, TID[name], TID_SCALE[name], fp8_e0(shape, name), cols, 0, q.numel(),
+                            factor_of(shape, name), q.data_ptr(), stream)
+    if rc == 0:
+        rc = lib.gen_fp8_scales_device(shape.seed, TID_SCALE[name], fp8_e0(shape, name), 0, sc.numel(),
+                                       sc.data_ptr(), stream)
+    if rc != 0:
+        raise RuntimeError(f"device FP8 generator failed for {name}: cudaError {rc}")
+    return q, sc
+
+
 def device_all(shape: LayerShape, device="cuda") -> dict:
-    names = ["x", "W_r", "W1", "W3", "W2"] + (["Ws1", "Ws3", "Ws2"] if shape.n_shared else [])
-    out = {nm: device_tensor(shape, nm, device) for nm in names}
+    """Every tensor of the layer on the device; with FP8 expert weights each
+    of W1, W3, W2, Ws1, Ws3, Ws2 is a (codes, scales) pair."""
+    experts = ["W1", "W3", "W2"] + (["Ws1", "Ws3", "Ws2"] if shape.n_shared else [])
+    out = {nm: device_tensor(shape, nm, device) for nm in ("x", "W_r")}
+    for nm in experts:
+        out[nm] = device_fp8(shape, nm, device) if shape.wdtype == "fp8" else device_tensor(shape, nm, device)
     out["b"] = device_tensor(shape, "b", device) if shape.bias else None
     if shape.n_shared == 0:
         out.update(Ws1=None, Ws3=None, Ws2=None)

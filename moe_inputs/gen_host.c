@@ -26,6 +26,7 @@
 #include <stdint.h>
 #include <string.h>
 #include <pthread.h>
+#include <math.h>
 
 static inline uint64_t splitmix64_out(uint64_t z) {
   z += 0x9E3779B97F4A7C15ull;
@@ -108,6 +109,83 @@ void gen_normal(uint32_t seed, uint32_t tid, uint64_t offset, uint64_t n, double
 void gen_uniform(uint32_t seed, uint32_t tid, uint64_t offset, uint64_t n, double lo, double hi,
                  int out_bf16, void* out, int nthreads) {
   run(seed, tid, 1, (uint32_t)out_bf16, offset, n, lo, hi, out, nthreads);
+}
+
+/*
+ * FP8 (e4m3) weights with one power-of-two scale per 128 x 128 block.
+ * For element i of a [rows, cols] matrix (flat row-major index i, cols a
+ * multiple of 128): block b = (r / 128) * (cols / 128) + c / 128 has the
+ * exponent e_b = e0 + (hash(seed, tid_scale, b) & 3); the code is the
+ * e4m3 value nearest (ties to even) to v_i * 2^-e_b, v_i the approximately
+ * normal value above (before any rounding), saturated to +-448. The scale
+ * byte of block b is e_b + 127 (UE8M0: value 2^(byte - 127)).
+ * e4m3: 1 sign, 4 exponent (bias 7), 3 mantissa bits; no infinities;
+ * 0x7F / 0xFF are NaN and never produced; largest finite 0x7E = 448.
+ */
+static inline uint8_t e4m3_rne(double x) {
+  uint8_t sign = (x < 0.0) ? 0x80 : 0x00;
+  double a = x < 0.0 ? -x : x;
+  if (a >= 464.0) return (uint8_t)(sign | 0x7E);            /* saturate (never reached here) */
+  if (a < 0.015625) {                                         /* below 2^-6: subnormal steps of 2^-9 */
+    int m = (int)rint(a * 512.0);                             /* exact scaling, ties to even */
+    return (uint8_t)(sign | m);                               /* m == 8 is the smallest normal, 0x08 */
+  }
+  int e;
+  double f = frexp(a, &e);                                    /* a = f 2^e, f in [0.5, 1) */
+  e -= 1;                                                     /* a = (2 f) 2^e, 2 f in [1, 2) */
+  int mant = (int)rint((ldexp(f, 1) - 1.0) * 8.0);
+  if (mant == 8) { mant = 0; e += 1; }
+  if (e > 8 || (e == 8 && mant > 6)) return (uint8_t)(sign | 0x7E);
+  return (uint8_t)(sign | ((e + 7) << 3) | mant);
+}
+
+static inline int block_exp(uint32_t seed, uint32_t tid_scale, uint64_t block, int e0) {
+  return e0 + (int)(splitmix64_out(gen_counter(seed, tid_scale, block)) & 3u);
+}
+
+typedef struct {
+  uint32_t seed, tid, tid_scale;
+  int e0;
+  uint64_t cols, offset, begin, end;
+  double factor;
+  uint8_t* out;
+} fp8_job_t;
+
+static void* run_fp8_job(void* p) {
+  fp8_job_t* j = (fp8_job_t*)p;
+  const uint64_t bcols = j->cols / 128;
+  for (uint64_t i = j->begin; i < j->end; ++i) {
+    const uint64_t g = j->offset + i, r = g / j->cols, c = g % j->cols;
+    const int e = block_exp(j->seed, j->tid_scale, (r / 128) * bcols + c / 128, j->e0);
+    const double v = irwin_hall4(splitmix64_out(gen_counter(j->seed, j->tid, g)), j->factor);
+    j->out[i] = e4m3_rne(ldexp(v, -e));
+  }
+  return 0;
+}
+
+/* e4m3 codes of elements [offset, offset + n) of a [rows, cols] matrix. */
+void gen_fp8(uint32_t seed, uint32_t tid, uint32_t tid_scale, int e0, uint64_t cols, uint64_t offset, uint64_t n,
+             double factor, uint8_t* out, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  if (n < (uint64_t)nthreads * 65536ull) nthreads = (int)(n / 65536ull) + 1;
+  fp8_job_t jobs[256];
+  pthread_t th[256];
+  uint64_t chunk = (n + nthreads - 1) / nthreads;
+  for (int t = 0; t < nthreads; ++t) {
+    uint64_t b0 = chunk * t, b1 = b0 + chunk;
+    if (b0 > n) b0 = n;
+    if (b1 > n) b1 = n;
+    jobs[t] = (fp8_job_t){seed, tid, tid_scale, e0, cols, offset, b0, b1, factor, out};
+  }
+  for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], 0, run_fp8_job, &jobs[t]);
+  run_fp8_job(&jobs[0]);
+  for (int t = 1; t < nthreads; ++t) pthread_join(th[t], 0);
+}
+
+/* UE8M0 scale bytes of blocks [offset, offset + n). */
+void gen_fp8_scales(uint32_t seed, uint32_t tid_scale, int e0, uint64_t offset, uint64_t n, uint8_t* out) {
+  for (uint64_t i = 0; i < n; ++i) out[i] = (uint8_t)(block_exp(seed, tid_scale, offset + i, e0) + 127);
 }
 
 /* Raw 64-bit hashes (used by the tests to pin the definition, and for seeded permutations). */

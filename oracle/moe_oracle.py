@@ -267,6 +267,36 @@ def forward(x: np.ndarray, W_r: np.ndarray, b, cfg: RouterCfg, expert, shared=No
     return y_routed + y_shared, routing, idx, gates
 
 
+# ---------------------------------------------------- FP8 expert weights ----
+
+def e4m3_value(codes: np.ndarray) -> np.ndarray:
+    """Value of OCP FP8 E4M3 codes (the element format of the FP8 checkpoint
+    the "DeepSeek-V3.2-Exp · Mixture of experts" page's Parameters section
+    mentions; format from the OCP 8-bit floating point specification):
+    1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0
+    holds subnormals m 2^-9; no infinities; 0x7F and 0xFF are NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return sign * mag
+
+
+def dequant_fp8(codes: np.ndarray, scales: np.ndarray, block: int = 128) -> np.ndarray:
+    """w[r, c] = e4m3(codes[r, c]) * 2^(scales[r // block, c // block] - 127),
+    exactly, in fp64: one UE8M0 (power-of-two) scale per block x block tile.
+    The pages say only that the checkpoint carries FP8 block scales; the block
+    size (128 x 128) and the scale format are DeepSeek-V3's."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    R, C = codes.shape
+    assert R % block == 0 and C % block == 0 and scales.shape == (R // block, C // block)
+    values = e4m3_value(np.arange(256, dtype=np.uint8))[codes]        # the code table, indexed
+    factors = np.exp2(np.asarray(scales, dtype=np.float64) - 127.0)   # exact powers of two
+    return (values.reshape(R // block, block, C // block, block) * factors[:, None, :, None]).reshape(R, C)
+
+
 # ------------------------------------------------- counts the pages print ----
 
 def expert_params(d: int, d_ff: int) -> int:

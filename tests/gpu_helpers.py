@@ -159,8 +159,8 @@ class PrefetchedExperts:
     so only a few experts are resident). Experts outside the order, or asked
     for again, are built on the spot."""
 
-    def __init__(self, s: mi.LayerShape, order, depth: int = 6):
-        self.fn = host_expert_fn(s)
+    def __init__(self, s: mi.LayerShape, order, depth: int = 6, fn=None):
+        self.fn = host_expert_fn(s) if fn is None else fn
         self.order = list(order)
         self.pos = {e: i for i, e in enumerate(self.order)}
         self.pool = concurrent.futures.ThreadPoolExecutor(max_workers=depth)

@@ -117,3 +117,65 @@ def test_device_generator_matches_host():
             dev = dev.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else dev.numpy()
             host = mi.host_tensor(s, nm, 0, n)
             assert (dev == host).all(), (name, nm)
+
+
+def _e4m3_nearest(x):
+    """Nearest finite E4M3 code to x by brute force over the code table, ties
+    to the even code (the one whose mantissa LSB is 0), saturating at 448."""
+    vals = []
+    for c in range(0x7F):
+        e, m = c >> 3, c & 7
+        vals.append(m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+    vals = np.array(vals)
+    a = min(abs(x), 448.0)
+    d = np.abs(vals - a)
+    best = np.flatnonzero(d == d.min())
+    c = int(best[0]) if len(best) == 1 else int([b for b in best if b % 2 == 0][0])
+    return c | (0x80 if x < 0 else 0)
+
+
+def test_fp8_generator_matches_definition():
+    # codes: nearest e4m3 to v * 2^-e_b with the block exponent from the
+    # scale tensor's hash; scales: e_b + 127
+    s = mi.SHAPES["v3_prefill_fp8"]
+    nm = "W1"
+    rows, cols = mi.mat_dims(s, nm)
+    e0 = mi.fp8_e0(s, nm)
+    idx = np.concatenate([np.arange(0, 300), np.arange(5 * cols + 100, 5 * cols + 400),
+                          np.arange(200 * cols + 7000, 200 * cols + 7168)])
+    codes = np.concatenate([mi.host_fp8(s, nm, int(i), 1) for i in idx])
+    factor = mi.factor_of(s, nm)
+    for i, code in zip(idx.tolist(), codes.tolist()):
+        h = mi.host_hash(s.seed, mi.TID[nm], i, 1)[0]
+        sm = int(h & 0xFFFF) + int((h >> 16) & 0xFFFF) + int((h >> 32) & 0xFFFF) + int(h >> 48)
+        v = float(sm - 131070) * factor
+        r, c = divmod(i, cols)
+        blk = (r // 128) * (cols // 128) + c // 128
+        eb = e0 + int(mi.host_hash(s.seed, mi.TID_SCALE[nm], blk, 1)[0] & 3)
+        assert code == _e4m3_nearest(math.ldexp(v, -eb)), (i, hex(code))
+        assert int(mi.host_fp8_scales(s, nm, blk, 1)[0]) == eb + 127
+    # the largest value the generator makes still fits: codes never saturate
+    assert 131070 * factor <= 448 * 2.0 ** e0
+
+
+def test_fp8_expert_slices_are_the_stacked_matrix():
+    s = mi.SHAPES["v3_decode_fp8"]
+    (q1, s1), _, (q2, s2) = mi.host_expert_fp8(s, 3)
+    F, d = s.d_ff, s.d
+    assert q1.shape == (F, d) and s1.shape == (F // 128, d // 128)
+    assert np.array_equal(q1[:2].reshape(-1), mi.host_fp8(s, "W1", 3 * F * d, 2 * d))
+    assert np.array_equal(s2.reshape(-1)[:5], mi.host_fp8_scales(s, "W2", 3 * (d // 128) * (F // 128), 5))
+
+
+@pytest.mark.gpu
+def test_device_fp8_generator_matches_host():
+    import torch
+    from moe_inputs import build, device
+    build.build_device()
+    s = mi.SHAPES["v3_decode_fp8"]
+    for nm in ("W1", "W2", "Ws2"):
+        q, sc = device.device_fp8(s, nm)
+        torch.cuda.synchronize()
+        n = min(q.numel(), 1 << 21)
+        assert np.array_equal(q.reshape(-1)[:n].cpu().numpy(), mi.host_fp8(s, nm, 0, n)), nm
+        assert np.array_equal(sc.reshape(-1).cpu().numpy(), mi.host_fp8_scales(s, nm)), nm

@@ -466,3 +466,43 @@ def test_bias_update_properties():
         assert np.allclose(np.abs(step[counts != mean]), 1e-3)
     # a perfectly balanced batch leaves the bias alone
     assert np.array_equal(oracle.bias_update(np.ones(8), np.full(8, 3), T=12, k=2, gamma=0.5), np.ones(8))
+
+
+# ------------------------------------------------------- FP8 weights ----
+
+def test_e4m3_code_values_from_the_format_definition():
+    # values fixed by the OCP FP8 E4M3 definition: zero, the smallest
+    # subnormal 2^-9, the largest subnormal 7 * 2^-9, the smallest normal
+    # 2^-6, one, 1.5, two, the largest finite 448, signs, NaN
+    table = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0, 0x3C: 1.5,
+             0x40: 2.0, 0x7E: 448.0, 0xFE: -448.0, 0xB8: -1.0, 0x80: -0.0,
+             0x4B: 5.5}  # 0x4B: exponent field 9 (2^2), mantissa 3 -> 1.375 * 4
+    for code, want in table.items():
+        got = oracle.e4m3_value(np.array([code], dtype=np.uint8))[0]
+        assert got == want and np.signbit(got) == np.signbit(want), (hex(code), got, want)
+    assert np.isnan(oracle.e4m3_value(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+    # the 127 non-negative finite codes are strictly increasing, spaced by the
+    # 3-bit mantissa step of their binade
+    v = oracle.e4m3_value(np.arange(0, 0x7F, dtype=np.uint8))
+    assert (np.diff(v) > 0).all()
+    assert np.allclose(np.diff(v)[:8], 2.0 ** -9)
+    # sign symmetry
+    pos = np.arange(0, 0x7F, dtype=np.uint8)
+    assert np.array_equal(oracle.e4m3_value(pos | 0x80), -v)
+
+
+def test_fp8_block_dequant_hand_example():
+    # a 128 x 256 matrix: two 128 x 128 blocks with scale bytes 127 (x1) and
+    # 125 (x1/4); code 0x40 (2.0) becomes 2.0 and 0.5, code 0xB8 (-1.0) becomes
+    # -1.0 and -0.25
+    codes = np.full((128, 256), 0x40, dtype=np.uint8)
+    codes[5, 7] = codes[9, 200] = 0xB8
+    scales = np.array([[127, 125]], dtype=np.uint8)
+    w = oracle.dequant_fp8(codes, scales)
+    assert w.shape == (128, 256)
+    assert w[0, 0] == 2.0 and w[127, 127] == 2.0 and w[0, 128] == 0.5 and w[127, 255] == 0.5
+    assert w[5, 7] == -1.0 and w[9, 200] == -0.25
+    # a 256 x 128 matrix with row blocks scaled by 2^3 and 2^-10
+    codes2 = np.full((256, 128), 0x38, dtype=np.uint8)
+    w2 = oracle.dequant_fp8(codes2, np.array([[130], [117]], dtype=np.uint8))
+    assert (w2[:128] == 8.0).all() and (w2[128:] == 2.0 ** -10).all()
