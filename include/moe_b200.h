@@ -314,6 +314,76 @@ MOE_API moe_status moe_bias_update(const moe_cfg* cfg, int64_t T, const int32_t*
                                    void* stream);
 
 /*
+ * Expert parallelism: the layer spread over W ranks (one process per GPU),
+ * rank r holding routed experts [r N / W, (r + 1) N / W) as in the page's
+ * quoted MoE.__init__ (experts sliced per rank), the router and the shared
+ * MLP on every rank. A rank's step (driven by the caller, who owns the
+ * all-to-all exchanges -- NCCL through torch.distributed in the package):
+ *   1. moe_route on its own tokens;
+ *   2. moe_dispatch_rows: expert histogram, expert-contiguous permutation,
+ *      the permuted token rows and their gates (rows for rank q's experts are
+ *      the contiguous range offsets[q E] .. offsets[(q + 1) E]);
+ *   3. exchange the per-expert counts and the rows (all-to-all);
+ *   4. moe_ep_reorder to expert-major order, moe_experts on the local
+ *      experts, moe_ep_reorder back;
+ *   5. exchange the gated rows back (all-to-all);
+ *   6. moe_experts for the shared MLP on its own tokens, then moe_combine.
+ * Every row is computed as in moe_forward, so each rank's y equals
+ * moe_forward's on the same tokens bit for bit.
+ */
+
+/*
+ * moe_dispatch plus the permuted rows: counts [N], offsets [N+1] (as
+ * moe_dispatch), slot_pos [T, top_k] (the permuted row of each of a token's
+ * experts, ascending expert; -1 for an invalid index), x_perm [T*top_k, d]
+ * (token rows in permuted order, cfg->dtype) and gate_perm [T*top_k] fp32
+ * (the gate of each permuted row, from gates [T, top_k]). All device
+ * buffers owned by the caller; workspace as for moe_workspace_size(cfg, T).
+ */
+MOE_API moe_status moe_dispatch_rows(const moe_cfg* cfg, int64_t T, const int32_t* topk_idx, const float* gates,
+                                     const void* x, int32_t* counts, int32_t* offsets, int32_t* slot_pos,
+                                     void* x_perm, float* gate_perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Grouped SwiGLU experts over rows already grouped by expert: the two
+ * tensor-core GEMMs of moe_forward (fp32 SIMT GEMMs for MOE_F32), without
+ * routing or combine. cfg supplies d, d_ff, dtype and n_routed = the number
+ * of groups E (1..512); its routing fields are ignored.
+ *   counts    [E] int32, device: rows of each group, in order; they must
+ *             sum to `rows` (checked on the device: otherwise no group is
+ *             computed and moe_device_status reports MOE_DEV_BAD_EXPERT)
+ *   x_rows    [rows, d]; gate_rows [rows] fp32 or NULL (gate 1)
+ *   W1, W3    [E, d_ff, d]; W2 [E, d, d_ff]
+ *   y_rows    [rows, d] out: gate * W2 (silu(W1 x) * W3 x) of each row
+ * Workspace: moe_experts_workspace_size(cfg, rows) bytes (the device-status
+ * word at its start is read by moe_device_status(cfg, rows, ...)).
+ */
+MOE_API moe_status moe_experts_workspace_size(const moe_cfg* cfg, int64_t rows, size_t* bytes);
+MOE_API moe_status moe_experts(const moe_cfg* cfg, int64_t rows, const int32_t* counts, const void* x_rows,
+                               const float* gate_rows, const void* W1, const void* W3, const void* W2, void* y_rows,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * y[t] = sum over the token's permuted rows slot_pos[t, 0..top_k)
+ * (ascending expert; -1 skipped) of routed_rows, plus shared_rows[t] (NULL
+ * for none), accumulated in fp32 in that order and rounded once.
+ *   routed_rows [T*top_k, d] in moe_dispatch_rows' permuted order
+ */
+MOE_API moe_status moe_combine(const moe_cfg* cfg, int64_t T, const void* routed_rows, const int32_t* slot_pos,
+                               const void* shared_rows, void* y, void* stream);
+
+/*
+ * Reorders rows between source-major order (blocks (p, e): rank p major,
+ * local expert e minor -- what an all-to-all delivers) and expert-major
+ * order (e major, p minor -- what moe_experts reads); to_expert_major
+ * selects the direction. counts [world, local_experts] int32, device: rows
+ * of each block. row_bytes must be a multiple of 4; src and dst 16-byte
+ * aligned, distinct buffers.
+ */
+MOE_API moe_status moe_ep_reorder(int32_t world, int32_t local_experts, const int32_t* counts, int64_t row_bytes,
+                                  const void* src, void* dst, int32_t to_expert_major, void* stream);
+
+/*
  * Self-check of the failure path (no counterpart in the pages): launches a
  * one-warp kernel that waits, with the same bounded wait every pipeline in
  * the library uses, on a barrier that nothing ever completes. After the wait

@@ -22,7 +22,8 @@ MOE_DEV_WAIT_TIMEOUT, MOE_DEV_BAD_EXPERT, MOE_DEV_DUP_EXPERT, MOE_DEV_TMEM_ALLOC
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE"}
 EXPORTS = ["moe_workspace_size", "moe_workspace_size_host", "moe_route", "moe_dispatch", "moe_forward",
-           "moe_forward_fp8",
+           "moe_forward_fp8", "moe_dispatch_rows", "moe_experts_workspace_size", "moe_experts", "moe_combine",
+           "moe_ep_reorder",
            "moe_forward_host", "moe_workspace_release", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update", "moe_selftest_wait_timeout",
            "moe_status_string", "moe_last_cuda_error"]
 STAGES = ["router", "dispatch", "gather", "gemm_swiglu", "gemm_gate", "combine"]
@@ -72,6 +73,11 @@ def lib() -> ctypes.CDLL:
         L.moe_route.argtypes = [CFG, I64, P, P, P, P, P, P, SZ, P]
         L.moe_dispatch.argtypes = [CFG, I64, P, P, P, P, P, SZ, P]
         L.moe_forward.argtypes = [CFG, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_dispatch_rows.argtypes = [CFG, I64, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_experts_workspace_size.argtypes = [CFG, I64, ctypes.POINTER(SZ)]
+        L.moe_experts.argtypes = [CFG, I64, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_combine.argtypes = [CFG, I64, P, P, P, P, P]
+        L.moe_ep_reorder.argtypes = [ctypes.c_int32, ctypes.c_int32, P, I64, P, P, ctypes.c_int32, P]
         FP8P = ctypes.POINTER(Fp8Matrix)
         L.moe_forward_fp8.argtypes = [CFG, I64, P, P, P, FP8P, FP8P, FP8P, FP8P, FP8P, FP8P, P, P, P, P, SZ, P]
         L.moe_forward_host.argtypes = [CFG, I64, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -209,6 +215,41 @@ def forward_fp8(cfg, T, x, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y, ws, topk_idx_ou
                                                     _fp8(W3), _fp8(W2), _fp8(Ws1), _fp8(Ws3), _fp8(Ws2), _ptr(y),
                                                     _ptr(topk_idx_out), _ptr(gates_out), _ptr(ws), ws_bytes,
                                                     _stream(stream)))
+
+
+def dispatch_rows(cfg, T, topk_idx, gates, x, counts, offsets, slot_pos, x_perm, gate_perm, ws, ws_bytes=None,
+                  stream=None):
+    """moe_dispatch plus the permuted token rows and their gates (expert parallelism, step 2)."""
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    _check("moe_dispatch_rows", lib().moe_dispatch_rows(ctypes.byref(cfg), T, _ptr(topk_idx), _ptr(gates), _ptr(x),
+                                                        _ptr(counts), _ptr(offsets), _ptr(slot_pos), _ptr(x_perm),
+                                                        _ptr(gate_perm), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def experts_workspace_size(cfg: MoeCfg, rows: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_experts_workspace_size", lib().moe_experts_workspace_size(ctypes.byref(cfg), rows, ctypes.byref(n)))
+    return n.value
+
+
+def experts(cfg, rows, counts, x_rows, gate_rows, W1, W3, W2, y_rows, ws, ws_bytes=None, stream=None):
+    """Grouped SwiGLU experts over rows grouped by expert (counts[e] rows each, in order)."""
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    _check("moe_experts", lib().moe_experts(ctypes.byref(cfg), rows, _ptr(counts), _ptr(x_rows), _ptr(gate_rows),
+                                            _ptr(W1), _ptr(W3), _ptr(W2), _ptr(y_rows), _ptr(ws), ws_bytes,
+                                            _stream(stream)))
+
+
+def combine(cfg, T, routed_rows, slot_pos, shared_rows, y, stream=None):
+    """y[t] = sum of the token's permuted rows (ascending expert) + shared_rows[t] (None for none)."""
+    _check("moe_combine", lib().moe_combine(ctypes.byref(cfg), T, _ptr(routed_rows), _ptr(slot_pos),
+                                            _ptr(shared_rows), _ptr(y), _stream(stream)))
+
+
+def ep_reorder(world, local_experts, counts, row_bytes, src, dst, to_expert_major, stream=None):
+    """Rows between source-major and expert-major order of the blocks counts[world, local_experts]."""
+    _check("moe_ep_reorder", lib().moe_ep_reorder(world, local_experts, _ptr(counts), row_bytes, _ptr(src), _ptr(dst),
+                                                  int(bool(to_expert_major)), _stream(stream)))
 
 
 def forward_host(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, ws_bytes=None,

@@ -55,29 +55,30 @@ struct Io<float> {
 // dispatch), -1 for a pair that was never placed.
 template <typename TE, int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_rows,
+                                                      const uint4* __restrict__ shared_rows,
                                                       const int32_t* __restrict__ slot_pos, int64_t T,
-                                                      int k, int has_shared, int64_t R, int vecs,
-                                                      uint4* __restrict__ y) {
+                                                      int k, int64_t R, int vecs, uint4* __restrict__ y) {
   constexpr int P = Io<TE>::kPerVec;
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    int32_t rows[KMAX + 1];  // row indices < R + T < 2^31
+    int32_t rows[KMAX];  // routed row indices < R < 2^31
 #pragma unroll
     for (int s = 0; s < KMAX; ++s) {
       const int32_t pos = s < k ? __ldg(slot_pos + t * k + s) : -1;
       rows[s] = (pos >= 0 && pos < R) ? pos : -1;
     }
-    rows[KMAX] = has_shared ? (int32_t)(R + t) : -1;
     for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
       uint4 buf[KMAX + 1];
 #pragma unroll
-      for (int s = 0; s < KMAX + 1; ++s)
+      for (int s = 0; s < KMAX; ++s)
         if (rows[s] >= 0) buf[s] = __ldg(y_rows + (int64_t)rows[s] * vecs + v);
+      if (shared_rows) buf[KMAX] = __ldg(shared_rows + t * vecs + v);
       float acc[P];
 #pragma unroll
       for (int i = 0; i < P; ++i) acc[i] = 0.f;
 #pragma unroll
-      for (int s = 0; s < KMAX + 1; ++s)
+      for (int s = 0; s < KMAX; ++s)
         if (rows[s] >= 0) Io<TE>::add(buf[s], acc);
+      if (shared_rows) Io<TE>::add(buf[KMAX], acc);
       y[t * vecs + v] = Io<TE>::pack(acc);
     }
   }
@@ -85,27 +86,34 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
 
 }  // namespace
 
-cudaError_t launch_combine(const Problem& p, const void* y_rows, const int32_t* slot_pos, void* y,
-                           cudaStream_t s) {
+cudaError_t launch_combine_rows(const Problem& p, const void* routed_rows, const void* shared_rows,
+                                const int32_t* slot_pos, void* y, cudaStream_t s) {
   const int vecs = (int)((int64_t)p.d * p.elem / 16);
   const int threads = vecs >= 256 ? 256 : (vecs >= 128 ? 128 : 64);
   int64_t cap = (int64_t)device_sm_count() * 16;
   unsigned blocks = (unsigned)(p.T < cap ? p.T : cap);
-  const uint4* yr = (const uint4*)y_rows;
-  const int sh = p.ns > 0;
+  const uint4* yr = (const uint4*)routed_rows;
+  const uint4* ys = (const uint4*)shared_rows;
   if (p.dtype == MOE_BF16) {
     if (p.k <= 8)
-      combine_kernel<__nv_bfloat16, 8><<<blocks, threads, 0, s>>>(yr, slot_pos, p.T, p.k, sh, p.R, vecs, (uint4*)y);
+      combine_kernel<__nv_bfloat16, 8><<<blocks, threads, 0, s>>>(yr, ys, slot_pos, p.T, p.k, p.R, vecs, (uint4*)y);
     else
-      combine_kernel<__nv_bfloat16, kMaxTopK><<<blocks, threads, 0, s>>>(yr, slot_pos, p.T, p.k, sh, p.R, vecs,
+      combine_kernel<__nv_bfloat16, kMaxTopK><<<blocks, threads, 0, s>>>(yr, ys, slot_pos, p.T, p.k, p.R, vecs,
                                                                         (uint4*)y);
   } else {
     if (p.k <= 8)
-      combine_kernel<float, 8><<<blocks, threads, 0, s>>>(yr, slot_pos, p.T, p.k, sh, p.R, vecs, (uint4*)y);
+      combine_kernel<float, 8><<<blocks, threads, 0, s>>>(yr, ys, slot_pos, p.T, p.k, p.R, vecs, (uint4*)y);
     else
-      combine_kernel<float, kMaxTopK><<<blocks, threads, 0, s>>>(yr, slot_pos, p.T, p.k, sh, p.R, vecs, (uint4*)y);
+      combine_kernel<float, kMaxTopK><<<blocks, threads, 0, s>>>(yr, ys, slot_pos, p.T, p.k, p.R, vecs, (uint4*)y);
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const Problem& p, const void* y_rows, const int32_t* slot_pos, void* y,
+                           cudaStream_t s) {
+  // y_rows: the R gated routed rows, then (with a shared MLP) its T rows
+  const void* shared = p.ns > 0 ? static_cast<const uint8_t*>(y_rows) + p.R * (int64_t)p.d * p.elem : nullptr;
+  return launch_combine_rows(p, y_rows, shared, slot_pos, y, s);
 }
 
 }  // namespace moe

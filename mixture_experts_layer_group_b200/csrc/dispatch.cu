@@ -237,7 +237,63 @@ __global__ void __launch_bounds__(256) gather_kernel(const TV* __restrict__ x,
   }
 }
 
+// Expert-parallel exchange order. counts [W, E]: rows that source rank p
+// sends for local expert e. Source-major order holds the blocks (p, e) as
+// p-major, e-minor (what an all-to-all delivers); expert-major order holds
+// them e-major, p-minor (what the grouped GEMMs read). One CTA per block
+// copies its rows, 16 or 4 bytes at a time.
+__global__ void __launch_bounds__(256) ep_reorder_kernel(const int32_t* __restrict__ counts, int W, int E,
+                                                         int64_t row_bytes, const uint8_t* __restrict__ src,
+                                                         uint8_t* __restrict__ dst, int to_expert_major) {
+  const int blk = blockIdx.x;
+  if (blk >= W * E) return;
+  const int p = blk / E, e = blk % E;
+  __shared__ int64_t offs[2];
+  if (threadIdx.x == 0) {
+    int64_t so = 0, eo = 0;
+    for (int q = 0; q < W; ++q)
+      for (int f = 0; f < E; ++f) {
+        const int64_t c = counts[q * E + f];
+        if (q < p || (q == p && f < e)) so += c;
+        if (f < e || (f == e && q < p)) eo += c;
+      }
+    offs[0] = so;
+    offs[1] = eo;
+  }
+  __syncthreads();
+  const int64_t n = counts[p * E + e];
+  const int64_t from = to_expert_major ? offs[0] : offs[1];
+  const int64_t to = to_expert_major ? offs[1] : offs[0];
+  const uint8_t* s = src + from * row_bytes;
+  uint8_t* d = dst + to * row_bytes;
+  const int64_t bytes = n * row_bytes;
+  if (row_bytes % 16 == 0) {
+    for (int64_t i = threadIdx.x; i < bytes / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(d)[i] = reinterpret_cast<const uint4*>(s)[i];
+  } else {
+    for (int64_t i = threadIdx.x; i < bytes / 4; i += blockDim.x)
+      reinterpret_cast<uint32_t*>(d)[i] = reinterpret_cast<const uint32_t*>(s)[i];
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_ep_reorder(const int32_t* counts, int W, int E, int64_t row_bytes, const void* src, void* dst,
+                              bool to_expert_major, cudaStream_t s) {
+  if (W <= 0 || E <= 0) return cudaSuccess;
+  ep_reorder_kernel<<<W * E, 256, 0, s>>>(counts, W, E, row_bytes, static_cast<const uint8_t*>(src),
+                                         static_cast<uint8_t*>(dst), to_expert_major ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unit_tables(const Problem& p, const int32_t* counts, const DispatchBuffers& db, int bm, int bn1,
+                               int bn2, cudaStream_t s) {
+  // the scan over a single "chunk" whose counts are the groups' row counts
+  ScanArgs sa{const_cast<int32_t*>(counts), 1, p.T, p.N, p.ns, p.F, p.nsF, p.d, bm, bn1, bn2,
+              db.counts, db.offsets, db.grp_row0, db.grp_rows, db.unit_base1, db.unit_base2};
+  scan_kernel<<<1, 1024, 0, s>>>(sa, db.chunk_base);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_dispatch(const Problem& p, const DispatchBuffers& db, int bm, int bn1, int bn2,
                             cudaStream_t s) {

@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kThreads) expert_gemm_simt_kernel(SimtParams p
       if (r >= rows_here) continue;
       const int64_t row = row0 + (int64_t)m * kBM + r;
       float* out = shared ? p.out_shared + row * p.ld_shared : p.out_routed + row * p.ld_routed;
-      const float gate = (kSwiGLU || shared) ? 1.f : p.gate_perm[row];
+      const float gate = (kSwiGLU || shared || !p.gate_perm) ? 1.f : p.gate_perm[row];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int c = tx + 16 * j;

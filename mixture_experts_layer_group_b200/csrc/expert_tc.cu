@@ -661,7 +661,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
           const int64_t row = row_base + tok;
           // gate of this lane's token, spread to the lanes that hold it below
           float my_gate = 1.0f;
-          if (MODE == kGateDown && !shared && tok < un.ntok) my_gate = __ldg(p.gate_perm + row);
+          if (MODE == kGateDown && !shared && p.gate_perm && tok < un.ntok) my_gate = __ldg(p.gate_perm + row);
           // The block (32 features = this quadrant's TMEM lanes, x 32 tokens =
           // columns j0..j0+31) in the m16n8 layout: lane half hf and column
           // group r give this thread features 16 hf + 8 e + lane / 4 (e = 0, 1)

@@ -98,6 +98,17 @@ cudaError_t launch_router(const Problem& p, const void* x, const void* W_r, cons
 cudaError_t launch_dispatch(const Problem& p, const DispatchBuffers& db, int bm, int bn1, int bn2,
                             cudaStream_t s);
 
+// Unit tables of the grouped GEMMs straight from per-group row counts
+// [p.N] (groups in order, rows contiguous): counts, offsets, grp_row0,
+// grp_rows and unit bases in db; db.chunk_base needs p.N ints of scratch.
+cudaError_t launch_unit_tables(const Problem& p, const int32_t* counts, const DispatchBuffers& db, int bm, int bn1,
+                               int bn2, cudaStream_t s);
+
+// Expert-parallel row reorder between source-major and expert-major order
+// of the blocks counts[W, E] (see ep_reorder_kernel).
+cudaError_t launch_ep_reorder(const int32_t* counts, int W, int E, int64_t row_bytes, const void* src, void* dst,
+                              bool to_expert_major, cudaStream_t s);
+
 // x_perm[slot_pos[t, s]] = x[t] for every placed (token, slot) pair
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* slot_pos, void* x_perm,
                           cudaStream_t s);
@@ -146,6 +157,9 @@ cudaError_t launch_expert_gemms_simt(const Problem& p, const GemmArgs& a, cudaSt
 // y_rows, plus the shared row y_rows[R + t]
 cudaError_t launch_combine(const Problem& p, const void* y_rows, const int32_t* slot_pos, void* y,
                            cudaStream_t s);
+// The same with the routed rows [R, d] and the shared rows [T, d] (or null) apart.
+cudaError_t launch_combine_rows(const Problem& p, const void* routed_rows, const void* shared_rows,
+                                const int32_t* slot_pos, void* y, cudaStream_t s);
 
 int device_sm_count();
 

@@ -321,6 +321,84 @@ moe_status check_weights(const Problem& p, const void* W_r, const float* b, cons
   return MOE_OK;
 }
 
+// moe_experts: a problem of E groups over `rows` grouped rows (no routing,
+// no shared MLP); workspace regions and a device check of the counts.
+moe_status make_group_problem(const moe_cfg* cfg, int64_t rows, Problem* p) {
+  if (!cfg || !p || rows < 0) return MOE_ERR_INVALID_ARG;
+  const moe_cfg& c = *cfg;
+  if (c.d <= 0 || c.d_ff <= 0 || c.n_routed <= 0 || c.d % 8 || c.d_ff % 8) return MOE_ERR_INVALID_ARG;
+  if (c.dtype != MOE_F32 && c.dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c.n_routed > kMaxRouted || (int64_t)c.n_routed * c.d_ff > (1ll << 31) ||
+      (int64_t)c.n_routed * c.d > (1ll << 31) || rows > (1ll << 31) - 1)
+    return MOE_ERR_UNSUPPORTED;
+  Problem q{};
+  q.T = rows;
+  q.d = c.d;
+  q.F = c.d_ff;
+  q.N = c.n_routed;
+  q.ns = 0;
+  q.k = 1;
+  q.G = 1;
+  q.TG = 1;
+  q.dtype = c.dtype;
+  q.R = rows;
+  q.nsF = 0;
+  q.elem = c.dtype == MOE_BF16 ? 2 : 4;
+  *p = q;
+  return MOE_OK;
+}
+
+struct GroupLayout {
+  size_t status, sched, counts_in, chunk_base, counts, offsets, grp_row0, grp_rows, unit_base1, unit_base2, h;
+  size_t total;
+};
+
+GroupLayout make_group_layout(const Problem& p) {
+  GroupLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  const size_t N = (size_t)p.N;
+  L.status = take(256);
+  L.sched = take(256);
+  L.counts_in = take(N * 4);
+  L.chunk_base = take(N * 4);
+  L.counts = take(N * 4);
+  L.offsets = take((N + 1) * 4);
+  L.grp_row0 = take((N + 1) * 4);
+  L.grp_rows = take((N + 1) * 4);
+  L.unit_base1 = take((N + 2) * 4);
+  L.unit_base2 = take((N + 2) * 4);
+  L.h = take((size_t)p.R * p.F * p.elem);
+  L.total = off;
+  return L;
+}
+
+// Copies the group counts into the workspace if they are non-negative and
+// sum to `rows`; otherwise writes zeros (no group runs) and flags the status.
+__global__ void check_counts_kernel(const int32_t* __restrict__ counts, int E, int64_t rows, int32_t* out,
+                                    unsigned* status) {
+  __shared__ unsigned long long total;
+  __shared__ int bad;
+  if (threadIdx.x == 0) {
+    total = 0;
+    bad = 0;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int32_t c = counts[e];
+    if (c < 0) atomicExch(&bad, 1);
+    atomicAdd(&total, (unsigned long long)(c < 0 ? 0 : c));
+  }
+  __syncthreads();
+  const bool ok = !bad && total == (unsigned long long)rows;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) out[e] = ok ? counts[e] : 0;
+  if (threadIdx.x == 0 && !ok) set_status(status, MOE_DEV_BAD_EXPERT);
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -504,6 +582,115 @@ moe_status moe_workspace_release(const void* ws) {
   g_pipes.erase(it);
   if (cur >= 0) cudaSetDevice(cur);
   return MOE_OK;
+}
+
+moe_status moe_dispatch_rows(const moe_cfg* cfg, int64_t T, const int32_t* topk_idx, const float* gates,
+                             const void* x, int32_t* counts, int32_t* offsets, int32_t* slot_pos, void* x_perm,
+                             float* gate_perm, void* ws, size_t ws_bytes, void* stream) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!topk_idx || !gates || !x || !counts || !offsets || !slot_pos || !x_perm || !gate_perm) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+  Layout L = make_layout(p);
+  if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  DispatchBuffers db = dispatch_buffers(L, ws, topk_idx, gates);
+  db.counts = counts;
+  db.offsets = offsets;
+  db.slot_pos = slot_pos;
+  db.gate_perm = gate_perm;
+  const bool tc = p.dtype == MOE_BF16;
+  cudaError_t e = cudaMemsetAsync(db.status, 0, 4, s);
+  if (e == cudaSuccess)
+    e = launch_dispatch(p, db, tc ? kTcBM : kSimtBM, tc ? kTcBN1 : kSimtBN, tc ? kTcBN2 : kSimtBN, s);
+  if (e == cudaSuccess) e = launch_gather(p, x, slot_pos, x_perm, s);
+  if (e == cudaSuccess) e = note_device_use(ws, s);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status moe_experts_workspace_size(const moe_cfg* cfg, int64_t rows, size_t* bytes) {
+  Problem p;
+  moe_status st = make_group_problem(cfg, rows, &p);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = make_group_layout(p).total;
+  return MOE_OK;
+}
+
+moe_status moe_experts(const moe_cfg* cfg, int64_t rows, const int32_t* counts, const void* x_rows,
+                       const float* gate_rows, const void* W1, const void* W3, const void* W2, void* y_rows,
+                       void* ws, size_t ws_bytes, void* stream) {
+  Problem p;
+  moe_status st = make_group_problem(cfg, rows, &p);
+  if (st != MOE_OK) return st;
+  if (rows == 0) return MOE_OK;
+  if (!counts || !x_rows || !y_rows || !W1 || !W3 || !W2) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_rows) || !aligned16(y_rows) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2))
+    return MOE_ERR_INVALID_ARG;
+  if (gate_rows && (reinterpret_cast<uintptr_t>(gate_rows) & 3u)) return MOE_ERR_INVALID_ARG;
+  const GroupLayout L = make_group_layout(p);
+  if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned* status = at<unsigned>(ws, L.status);
+  cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  check_counts_kernel<<<1, 256, 0, s>>>(counts, p.N, rows, at<int32_t>(ws, L.counts_in), status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  DispatchBuffers db{};
+  db.chunk_base = at<int32_t>(ws, L.chunk_base);
+  db.counts = at<int32_t>(ws, L.counts);
+  db.offsets = at<int32_t>(ws, L.offsets);
+  db.grp_row0 = at<int32_t>(ws, L.grp_row0);
+  db.grp_rows = at<int32_t>(ws, L.grp_rows);
+  db.unit_base1 = at<int32_t>(ws, L.unit_base1);
+  db.unit_base2 = at<int32_t>(ws, L.unit_base2);
+  const bool tc = p.dtype == MOE_BF16;
+  e = launch_unit_tables(p, at<int32_t>(ws, L.counts_in), db, tc ? kTcBM : kSimtBM, tc ? kTcBN1 : kSimtBN,
+                         tc ? kTcBN2 : kSimtBN, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  GemmArgs ga;
+  ga.x = nullptr;
+  ga.x_perm = x_rows;
+  ga.W1 = W1;
+  ga.W3 = W3;
+  ga.W2 = W2;
+  ga.Ws1 = ga.Ws3 = ga.Ws2 = nullptr;
+  ga.h_perm = at<void>(ws, L.h);
+  ga.h_sh = nullptr;
+  ga.y_rows = y_rows;
+  ga.grp_row0 = db.grp_row0;
+  ga.grp_rows = db.grp_rows;
+  ga.unit_base1 = db.unit_base1;
+  ga.unit_base2 = db.unit_base2;
+  ga.gate_perm = gate_rows;
+  ga.status = status;
+  ga.sched = at<int>(ws, L.sched);
+  e = tc ? launch_expert_gemms_tc(p, ga, s, nullptr) : launch_expert_gemms_simt(p, ga, s, nullptr);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status moe_combine(const moe_cfg* cfg, int64_t T, const void* routed_rows, const int32_t* slot_pos,
+                       const void* shared_rows, void* y, void* stream) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!routed_rows || !slot_pos || !y || !aligned16(routed_rows) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (shared_rows && !aligned16(shared_rows)) return MOE_ERR_INVALID_ARG;
+  cudaError_t e = launch_combine_rows(p, routed_rows, shared_rows, slot_pos, y, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status moe_ep_reorder(int32_t world, int32_t local_experts, const int32_t* counts, int64_t row_bytes,
+                          const void* src, void* dst, int32_t to_expert_major, void* stream) {
+  if (world <= 0 || local_experts <= 0 || (int64_t)world * local_experts > (1 << 20) || row_bytes <= 0 ||
+      row_bytes % 4 || !counts || !src || !dst || src == dst || !aligned16(src) || !aligned16(dst))
+    return MOE_ERR_INVALID_ARG;
+  cudaError_t e = launch_ep_reorder(counts, world, local_experts, row_bytes, src, dst, to_expert_major != 0,
+                                    (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
 moe_status moe_device_status(const moe_cfg* cfg, int64_t T, void* ws, size_t ws_bytes, int clear,

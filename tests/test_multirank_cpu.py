@@ -113,3 +113,121 @@ def test_bench_gpus_2_starts_two_ranks():
     assert rep["n_gpus"] == 2
     assert sorted(r["rank"] for r in rep["ranks"]) == [0, 1]
     assert len({r["pid"] for r in rep["ranks"]}) == 2
+
+
+class _OracleOps:
+    """CPU stand-ins for the device steps of an expert-parallel rank (fp64,
+    from the oracle's definitions), so the exchange logic of the product's
+    ExpertParallelMoE can run over gloo without a GPU."""
+
+    def __init__(self, lc, E):
+        import oracle
+        self.o = oracle
+        self.lc, self.E = lc, E
+        self.rcfg = oracle.RouterCfg(n_routed=lc.n_routed, top_k=lc.top_k, score=lc.score, n_groups=lc.n_groups,
+                                     topk_groups=lc.topk_groups, normalize=lc.normalize,
+                                     route_scale=lc.route_scale, group_score=lc.group_score)
+
+    def route_dispatch(self, x, W_r, b):
+        import numpy as np
+        import torch
+        r = self.o.route(x.numpy(), W_r.numpy(), None if b is None else b.numpy(), self.rcfg)
+        counts, offsets, perm = self.o.permutation(r.idx, self.lc.n_routed)
+        k = self.lc.top_k
+        T = x.shape[0]
+        pos = np.empty(T * k, dtype=np.int64)
+        pos[perm] = np.arange(T * k)
+        slot_pos = np.empty((T, k), dtype=np.int64)
+        for t in range(T):  # the token's rows in ascending expert order
+            order = np.argsort(r.idx[t], kind="stable")
+            slot_pos[t] = pos[t * k + order]
+        x_perm = x[torch.from_numpy(perm // k)]
+        gate_perm = torch.from_numpy(r.gates.reshape(-1)[perm])
+        return (torch.from_numpy(counts.astype(np.int32)), torch.from_numpy(slot_pos), x_perm, gate_perm)
+
+    def reorder(self, W, block_counts, rows, to_expert_major):
+        import torch
+        c = block_counts.tolist()
+        src, o = {}, 0
+        for p in range(W):
+            for e in range(self.E):
+                src[(p, e)] = o
+                o += c[p][e]
+        em = [i for e in range(self.E) for p in range(W) for i in range(src[(p, e)], src[(p, e)] + c[p][e])]
+        idx = torch.tensor(em, dtype=torch.int64)
+        if to_expert_major:
+            return rows[idx]
+        out = torch.empty_like(rows)
+        out[idx] = rows
+        return out
+
+    def experts(self, counts, rows, gates, W1, W3, W2):
+        import torch
+        out = torch.empty_like(rows)
+        o = 0
+        for e, n in enumerate(counts.tolist()):
+            if n:
+                y = self.o.expert_ffn(rows[o:o + n].numpy(), W1[e].numpy(), W3[e].numpy(), W2[e].numpy())
+                out[o:o + n] = torch.from_numpy(y * gates[o:o + n].numpy()[:, None])
+            o += n
+        return out
+
+    def shared(self, x, Ws1, Ws3, Ws2):
+        import torch
+        return torch.from_numpy(self.o.expert_ffn(x.numpy(), Ws1.numpy(), Ws3.numpy(), Ws2.numpy()))
+
+    def combine(self, routed_rows, slot_pos, shared_rows):
+        y = routed_rows[slot_pos].sum(dim=1)
+        return y if shared_rows is None else y + shared_rows
+
+
+def _ep_worker(rank, world, port, out):
+    import datetime
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import oracle
+    from mixture_experts_layer_group_b200 import ep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank))
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        rng = np.random.default_rng(7)  # the same layer on every rank
+        N, d, F, k, ns = 12, 10, 8, 3, 1
+        W_r = rng.standard_normal((N, d)) / np.sqrt(d)
+        b = rng.uniform(-0.1, 0.1, N)
+        W1, W3 = rng.standard_normal((N, F, d)) / np.sqrt(d), rng.standard_normal((N, F, d)) / np.sqrt(d)
+        W2 = rng.standard_normal((N, d, F)) / np.sqrt(F)
+        Ws = (rng.standard_normal((ns * F, d)), rng.standard_normal((ns * F, d)), rng.standard_normal((d, ns * F)))
+        x = np.random.default_rng(100 + rank).standard_normal((20 + 5 * rank, d))  # own tokens per rank
+        lc = ep.LayerCfg(d, F, N, ns, k, n_groups=4, topk_groups=2, score="sigmoid", normalize=True,
+                         route_scale=2.5, dtype="f32")
+        E = N // world
+        t = torch.from_numpy
+        w = {"W_r": t(W_r), "b": t(b), "W1": t(W1[rank * E:(rank + 1) * E]), "W3": t(W3[rank * E:(rank + 1) * E]),
+             "W2": t(W2[rank * E:(rank + 1) * E]), "Ws1": t(Ws[0]), "Ws3": t(Ws[1]), "Ws2": t(Ws[2])}
+        layer = ep.ExpertParallelMoE(lc, rank, world, w, ops=_OracleOps(lc, E))
+        y = layer.forward(t(x)).numpy()
+        rcfg = _OracleOps(lc, E).rcfg
+        ref, *_ = oracle.forward(x, W_r, b, rcfg, lambda e: (W1[e], W3[e], W2[e]), Ws)
+        out.put((rank, float(np.abs(y - ref).max()), float(np.abs(ref).max())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_expert_parallel_exchange_over_gloo(world):
+    # each rank routes its own tokens, sends rows to the ranks holding their
+    # experts, computes its expert block, returns the rows and combines: the
+    # result is the oracle's whole-layer forward on that rank's tokens
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, err, scale in res:
+        assert err <= 1e-12 * max(scale, 1.0), (rank, err)
