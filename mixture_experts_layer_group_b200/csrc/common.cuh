@@ -304,6 +304,13 @@ MOE_DEV void umma_commit_pair(uint32_t bar_cluster) {
                : "memory");
 }
 
+// Arrives on the mbarrier at the same shared-memory offset in both CTAs of
+// the pair once the pair MMAs issued so far by this thread have completed.
+MOE_DEV void umma_commit_pair_both(uint32_t bar_smem) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               ::"r"(bar_smem), "h"((uint16_t)3) : "memory");
+}
+
 // Arrives on `bar` once every tcgen05 operation issued so far by this thread
 // has completed.
 MOE_DEV void umma_commit(uint64_t* bar) {

@@ -561,18 +561,13 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
             umma_bf16_pair(d0, smem_desc_sw128(a_addr + kk * 32), bdesc, idesc, (kc | kk) != 0);
             umma_bf16_pair(d1, smem_desc_sw128(a_addr + kHalfBytes + kk * 32), bdesc, idesc, (kc | kk) != 0);
           }
-          umma_commit_pair(smem_u32(&sh.empty[s]));
-          umma_commit_pair(peer(&sh.empty[s]));
-          if (FP8) {
-            umma_commit_pair(smem_u32(&shf.conv_empty[c]));
-            umma_commit_pair(peer(&shf.conv_empty[c]));
-          }
+          umma_commit_pair_both(smem_u32(&sh.empty[s]));
+          if (FP8) umma_commit_pair_both(smem_u32(&shf.conv_empty[c]));
         }
         if (ok) {
           for (int b = 0; b < 2; ++b)
             if ((mask >> b) & 1u) {
-              umma_commit_pair(smem_u32(&sh.acc_full[b]));
-              umma_commit_pair(peer(&sh.acc_full[b]));
+              umma_commit_pair_both(smem_u32(&sh.acc_full[b]));
             }
         }
       }
@@ -581,8 +576,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         set_status(p.status, MOE_DEV_WAIT_TIMEOUT);
       }
       // all pair MMAs have completed once `drained` fires (in both CTAs)
-      umma_commit_pair(smem_u32(&sh.drained));
-      umma_commit_pair(peer(&sh.drained));
+      umma_commit_pair_both(smem_u32(&sh.drained));
       sh.consumed = consumed;
     }
     if (lane == 0) {
