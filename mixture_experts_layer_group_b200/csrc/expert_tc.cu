@@ -75,11 +75,8 @@ constexpr int kATileBytes = 2 * kHalfBytes;       // 32 KB: this CTA's rows of b
 constexpr int kMaxStageBytes = kATileBytes + (kMaxTok / 2 / kTokBox) * kBoxBytes;  // 48 KB
 constexpr int kBufCols = 256;                     // fp32 columns per accumulator buffer
 constexpr int kTmemCols = 2 * kBufCols;           // 2 buffers
-constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant
-constexpr int kCvtWarps = 4;                      // FP8 weights: dequantising warps
 constexpr int kRing = 8;                          // unit ids in flight between the roles
 constexpr int kTileBytes = 32 * 32 * 2;           // a warp's dense 32 x 32 bf16 tile (TMA store box)
-constexpr int kTBytes = kEpiWarps * kTileBytes;        // one tile per epilogue warp
 constexpr int kA8Bytes = 2 * 128 * kBK;           // 16 KB: the fp8 codes of a CTA's 256 weight rows x 64 K
 constexpr int kFp8Block = 128;                    // FP8 scale block (rows and columns)
 
@@ -92,6 +89,8 @@ template <bool FP8>
 struct Plan;
 template <>
 struct Plan<false> {
+  static constexpr int kEpiWarps = 8;            // two per TMEM lane quadrant
+  static constexpr int kCvtWarps = 4;            // (no converters; 4 keeps the arithmetic defined)
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kRingBytes = 52 * 4096;   // 208 KB
   static constexpr int kABytes = kATileBytes;    // weight bytes at the head of a stage
@@ -101,6 +100,8 @@ struct Plan<false> {
 };
 template <>
 struct Plan<true> {
+  static constexpr int kEpiWarps = 8;            // two per TMEM lane quadrant
+  static constexpr int kCvtWarps = 4;            // dequantising warps
   static constexpr int kThreads = 64 + 32 * (kEpiWarps + kCvtWarps);
   static constexpr int kRingBytes = 36 * 4096;   // 144 KB
   static constexpr int kABytes = kA8Bytes;
@@ -109,14 +110,18 @@ struct Plan<true> {
   static constexpr int kBarrierBytes = 1024;
 };
 template <bool FP8>
+__host__ __device__ constexpr int tile_bytes() {
+  return Plan<FP8>::kEpiWarps * kTileBytes;  // one transpose tile per epilogue warp
+}
+template <bool FP8>
 constexpr int smem_bytes() {
-  return Plan<FP8>::kRingBytes + Plan<FP8>::kConvBytes + kTBytes + 1024 + Plan<FP8>::kBarrierBytes;
+  return Plan<FP8>::kRingBytes + Plan<FP8>::kConvBytes + tile_bytes<FP8>() + 1024 + Plan<FP8>::kBarrierBytes;
 }
 static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory budget");
 static_assert(kMaxStageBytes * 3 <= Plan<false>::kRingBytes, "ring holds three full stages");
 static_assert((kA8Bytes + (kMaxTok / 2 / kTokBox) * kBoxBytes) * 4 <= Plan<true>::kRingBytes,
               "FP8 ring holds four full stages");
-static_assert(kEpiWarps % 4 == 0, "whole quadrants");
+static_assert(Plan<false>::kEpiWarps % 4 == 0 && Plan<true>::kEpiWarps % 4 == 0, "whole quadrants");
 static_assert(kMaxTok <= kBufCols && kMaxTok % (2 * kTokBox) == 0, "token chunk");
 
 enum Mode : int { kSwiGLU = 0, kGateDown = 1 };
@@ -241,9 +246,11 @@ struct SharedFp8 {
 static_assert(512 + sizeof(SharedFp8) <= Plan<true>::kBarrierBytes, "FP8 barrier block");
 
 // Barrier among the epilogue warps only (id 1; id 0 is __syncthreads).
-MOE_DEV void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
+template <int kWarps>
+MOE_DEV void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kWarps) : "memory"); }
 // Barrier among the FP8 converter warps only (id 2).
-MOE_DEV void cvt_sync() { asm volatile("bar.sync 2, %0;" ::"n"(32 * kCvtWarps) : "memory"); }
+template <int kWarps>
+MOE_DEV void cvt_sync() { asm volatile("bar.sync 2, %0;" ::"n"(32 * kWarps) : "memory"); }
 
 // f16 pair -> the bf16 pair of its values times 2^-112, for f16 values
 // converted from e4m3: they carry 3 mantissa bits and are never f16
@@ -317,6 +324,7 @@ template <int MODE, bool FP8>
 __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
   using PL = Plan<FP8>;
   constexpr int kRingBytes = PL::kRingBytes;
+  constexpr int kEpiWarps = PL::kEpiWarps, kCvtWarps = PL::kCvtWarps, kTBytes = tile_bytes<FP8>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* conv = smem + kRingBytes;  // FP8: the dequantised weight slots
@@ -388,9 +396,11 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
       // launch): nothing it loads may be read before that grid has finished
       if (MODE == kGateDown) griddep_wait();
       // a weight tile read by one unit only is streamed once: evict it first;
-      // tiles shared by the chunks of a large group stay at normal priority
+      // tiles shared by the chunks of a large group, and the token rows (read
+      // by every feature tile of their group), are kept in L2 as long as possible
       const uint64_t pol_once = policy_evict_first();
       const uint64_t pol_shared = policy_evict_normal();
+      const uint64_t pol_last = policy_evict_last();
       // Ring allocation (identical in both CTAs, so stage offsets match).
       // Stages are placed back to back in fill order and freed in the same
       // order by the pair MMAs' commits, so the bytes in use form one circular
@@ -472,7 +482,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         const CUtensorMap* ta0 = shared ? &p.a0_shared : &p.a0_routed;
         const CUtensorMap* ta1 = MODE == kSwiGLU ? (shared ? &p.a1_shared : &p.a1_routed) : ta0;
         const CUtensorMap* tb = shared ? &p.b_shared[tmap] : &p.b_routed[tmap];
-        const uint64_t pol = un.nchunks == 1 ? pol_once : pol_shared;
+        const uint64_t pol = un.nchunks == 1 ? pol_once : pol_last;
         for (int kc = 0; kc < nk; ++kc, ++fills) {
           const uint32_t s = fills % kSlots;
           uint32_t pos = 0;
@@ -491,13 +501,13 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
             mbar_arrive_expect_tx(&sh.full[s], tx);
             tma_load_2d_hint(a_dst, ta0, &sh.full[s], kc * kBK, rowA, pol);
             if (MODE == kSwiGLU) tma_load_2d_hint(a_dst + kA8Bytes / 2, ta1, &sh.full[s], kc * kBK, rowA, pol);
-            tma_load_2d_hint(b_dst, tb, &sh.full[s], kc * kBK, rowB, pol_shared);
+            tma_load_2d_hint(b_dst, tb, &sh.full[s], kc * kBK, rowB, pol_last);
           } else {
             const uint32_t full_bar = in_first(&sh.full[s]);
             if (first) mbar_arrive_expect_tx(&sh.full[s], 2 * tx);  // this CTA's bytes and the peer's
             tma_load_2d_pair(a_dst, ta0, full_bar, kc * kBK, rowA, pol);  // SwiGLU: 128 W1 rows; down: 256 rows
             if (MODE == kSwiGLU) tma_load_2d_pair(a_dst + kHalfBytes, ta1, full_bar, kc * kBK, rowA, pol);
-            tma_load_2d_pair(b_dst, tb, full_bar, kc * kBK, rowB, pol_shared);
+            tma_load_2d_pair(b_dst, tb, full_bar, kc * kBK, rowB, pol_last);
           }
         }
         if (!ok) break;
@@ -624,7 +634,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         }
         sh.epi_unit[i & 1] = u;
       }
-      epi_sync();
+      epi_sync<kEpiWarps>();
       const int u = load_volatile(&sh.epi_unit[i & 1]);
       if (u < 0) break;
       Unit un;
@@ -772,7 +782,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         }
         shf.cvt_unit[i & 1] = u;
       }
-      cvt_sync();
+      cvt_sync<kCvtWarps>();
       if (load_volatile(&shf.cvt_unit[i & 1]) < 0) break;
       const int g = load_volatile(&shf.cvt_info[i & 1][0]);
       const int f = load_volatile(&shf.cvt_info[i & 1][1]);
@@ -806,7 +816,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
           }
           shf.cvt_ok = ok;
         }
-        cvt_sync();
+        cvt_sync<kCvtWarps>();
         if (!load_volatile(&shf.cvt_ok)) {
           alive = false;
           break;
@@ -835,7 +845,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
           st_shared_v4(row + (((2 * q4 + 1) ^ (rr & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
         }
         fence_proxy_async_smem();  // the tensor cores read the slot through the async proxy
-        cvt_sync();
+        cvt_sync<kCvtWarps>();
         if (cleader) {
           if (first) mbar_arrive(&shf.conv_full[c]);
           else mbar_arrive_cluster(in_first(&shf.conv_full[c]));
