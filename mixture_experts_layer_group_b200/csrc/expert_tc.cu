@@ -399,7 +399,6 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
       // tiles shared by the chunks of a large group, and the token rows (read
       // by every feature tile of their group), are kept in L2 as long as possible
       const uint64_t pol_once = policy_evict_first();
-      const uint64_t pol_shared = policy_evict_normal();
       const uint64_t pol_last = policy_evict_last();
       // Ring allocation (identical in both CTAs, so stage offsets match).
       // Stages are placed back to back in fill order and freed in the same
