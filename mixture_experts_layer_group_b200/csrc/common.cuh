@@ -116,6 +116,15 @@ MOE_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
+// 4-byte store into shared memory of a CTA of the cluster that completes 4
+// transaction bytes on an mbarrier of that CTA (its complete_tx has release
+// semantics at cluster scope). The issuing thread does not wait for it.
+MOE_DEV void st_async_u32(uint32_t cluster_addr, uint32_t v, uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(cluster_addr),
+               "r"(v), "r"(bar_cluster)
+               : "memory");
+}
+
 MOE_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -296,6 +305,21 @@ MOE_DEV void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, u
       : "memory");
 }
 
+// Pair MMA with A in tensor memory: D[256 x N] (+)= A[256 x 16] * B[N x 16]^T,
+// A rows 0..127 in this CTA's TMEM lanes 0..127 at column a_tmem (16 bf16
+// of a row packed two per 32-bit column, lower k in the low half) and rows
+// 128..255 at the same address in the peer's; B as in umma_bf16_pair.
+// N must be a multiple of 32.
+MOE_DEV void umma_bf16_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives on the mbarrier at cluster address `bar_cluster` (this CTA's or the
 // peer's) once the pair MMAs issued so far by this thread have completed.
 MOE_DEV void umma_commit_pair(uint32_t bar_cluster) {
@@ -386,6 +410,22 @@ MOE_DEV void stmatrix_x4_trans(uint32_t smem_addr, uint32_t r0, uint32_t r1, uin
 }
 
 MOE_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 32 consecutive 32-bit columns to tensor memory: thread i of the
+// warp writes r[0..31] to row (lane base + i). The caller issues
+// tmem_wait_st() before signalling that the columns are written.
+MOE_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+      " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+MOE_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------ values --
 

@@ -52,6 +52,12 @@
 //               shared-memory tile with stmatrix.trans and writes it with one
 //               TMA tensor store (a ragged last block with 64-byte row
 //               stores); no barrier between epilogue warps per block
+// With FP8 (e4m3) weights the same kernel runs 448 threads: the producer
+// loads the codes (64-byte swizzled rows) and the token box into the ring,
+// eight converter warps (one per TMEM lane quadrant and weight half)
+// dequantise each stage's codes exactly into bf16 in tensor memory, and the
+// pair MMAs read A from there and B from the ring (kind::f16 as above); four
+// epilogue warps, one per quadrant.
 // Every mbarrier wait is bounded; on a timeout a CTA records
 // MOE_DEV_WAIT_TIMEOUT, drains its own copies and MMAs (bounded again),
 // frees its tensor memory and exits.
@@ -72,19 +78,25 @@ constexpr int kBoxBytes = kTokBox * kBK * 2;      // 4 KB
 constexpr int kTokMaps = 3;                       // token boxes of 32, 64 and 128 rows
 constexpr int kHalfBytes = 128 * kBK * 2;         // 16 KB: 128 weight rows of one half
 constexpr int kATileBytes = 2 * kHalfBytes;       // 32 KB: this CTA's rows of both halves
-constexpr int kMaxStageBytes = kATileBytes + (kMaxTok / 2 / kTokBox) * kBoxBytes;  // 48 KB
-constexpr int kBufCols = 256;                     // fp32 columns per accumulator buffer
-constexpr int kTmemCols = 2 * kBufCols;           // 2 buffers
+constexpr int kMaxTokBytes = (kMaxTok / 2 / kTokBox) * kBoxBytes;  // 16 KB: a CTA's largest token box
+constexpr int kMaxStageBytes = kATileBytes + kMaxTokBytes;          // 48 KB
+constexpr int kTmemCols = 512;                    // the pair allocation in each CTA
 constexpr int kRing = 8;                          // unit ids in flight between the roles
 constexpr int kTileBytes = 32 * 32 * 2;           // a warp's dense 32 x 32 bf16 tile (TMA store box)
 constexpr int kA8Bytes = 2 * 128 * kBK;           // 16 KB: the fp8 codes of a CTA's 256 weight rows x 64 K
 constexpr int kFp8Block = 128;                    // FP8 scale block (rows and columns)
+constexpr int kASlots = 3;                        // FP8: dequantised weight stages in tensor memory
+constexpr int kASlotCols = 2 * kBK / 2;           // FP8: columns of one slot (two halves x 64 bf16 / 2)
 
-// Shared-memory plan. bf16 weights: one ring of variable-size stages (this
-// CTA's 256 weight rows x 64 K in bf16, then the token box). FP8 weights: the
-// ring holds the fp8 codes (16 KB) and the token box; the converter warps
-// write the dequantised bf16 weight tile of each stage into one of kConv
-// slots, which the MMAs read with the stage's token box.
+// Shared-memory and tensor-memory plan. bf16 weights: one ring of
+// variable-size stages (this CTA's 256 weight rows x 64 K in bf16, then the
+// token box), which the MMAs read in place; TMEM holds two accumulator
+// buffers of 256 columns. FP8 weights: the ring holds the fp8 codes (16 KB,
+// 64-byte swizzled rows) and the token box; the converter warps dequantise
+// each stage's codes in registers into one of two weight slots in tensor
+// memory (three slots, columns 320..511), from which the pair MMAs take A
+// (B, the token box, stays in the ring); the accumulators share columns
+// 0..319, so a unit covers at most 160 tokens.
 template <bool FP8>
 struct Plan;
 template <>
@@ -94,19 +106,21 @@ struct Plan<false> {
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kRingBytes = 52 * 4096;   // 208 KB
   static constexpr int kABytes = kATileBytes;    // weight bytes at the head of a stage
-  static constexpr int kConv = 1;                // (no conversion slots; 1 keeps the arithmetic defined)
-  static constexpr int kConvBytes = 0;
+  static constexpr int kChunk = kTcBM;           // token rows of a unit at most
+  static constexpr int kTokAlign = 16;           // MMA N granule
+  static constexpr uint32_t kAccCols = 512;      // accumulator columns: two buffers of 256
   static constexpr int kBarrierBytes = 512;
 };
 template <>
 struct Plan<true> {
-  static constexpr int kEpiWarps = 8;            // two per TMEM lane quadrant
-  static constexpr int kCvtWarps = 4;            // dequantising warps
+  static constexpr int kEpiWarps = 4;            // one per TMEM lane quadrant
+  static constexpr int kCvtWarps = 8;            // two per TMEM lane quadrant: one per weight half
   static constexpr int kThreads = 64 + 32 * (kEpiWarps + kCvtWarps);
-  static constexpr int kRingBytes = 36 * 4096;   // 144 KB
+  static constexpr int kRingBytes = 54 * 4096;   // 216 KB
   static constexpr int kABytes = kA8Bytes;
-  static constexpr int kConv = 2;
-  static constexpr int kConvBytes = kConv * kATileBytes;
+  static constexpr int kChunk = kTcBM8;
+  static constexpr int kTokAlign = 32;           // N of an MMA with A in tensor memory
+  static constexpr uint32_t kAccCols = 320;      // two buffers of 160; then the weight slots
   static constexpr int kBarrierBytes = 1024;
 };
 template <bool FP8>
@@ -115,14 +129,20 @@ __host__ __device__ constexpr int tile_bytes() {
 }
 template <bool FP8>
 constexpr int smem_bytes() {
-  return Plan<FP8>::kRingBytes + Plan<FP8>::kConvBytes + tile_bytes<FP8>() + 1024 + Plan<FP8>::kBarrierBytes;
+  return Plan<FP8>::kRingBytes + tile_bytes<FP8>() + 1024 + Plan<FP8>::kBarrierBytes;
 }
 static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory budget");
 static_assert(kMaxStageBytes * 3 <= Plan<false>::kRingBytes, "ring holds three full stages");
-static_assert((kA8Bytes + (kMaxTok / 2 / kTokBox) * kBoxBytes) * 4 <= Plan<true>::kRingBytes,
-              "FP8 ring holds four full stages");
+static_assert((kA8Bytes + kMaxTokBytes) * 4 <= Plan<true>::kRingBytes, "FP8 ring holds four full stages");
 static_assert(Plan<false>::kEpiWarps % 4 == 0 && Plan<true>::kEpiWarps % 4 == 0, "whole quadrants");
-static_assert(kMaxTok <= kBufCols && kMaxTok % (2 * kTokBox) == 0, "token chunk");
+static_assert(Plan<true>::kCvtWarps == 8, "one converter warp per (TMEM lane quadrant, weight half)");
+static_assert(2 * Plan<false>::kChunk <= (int)Plan<false>::kAccCols && 2 * Plan<true>::kChunk <= (int)Plan<true>::kAccCols &&
+                  Plan<true>::kAccCols % 64 == 0 &&
+                  Plan<true>::kAccCols + kASlots * kASlotCols <= (uint32_t)kTmemCols,
+              "accumulators and weight slots fit the tensor memory");
+static_assert(kMaxTok % (2 * kTokBox) == 0 && Plan<false>::kChunk <= kMaxTok && Plan<true>::kChunk <= kMaxTok &&
+                  Plan<true>::kChunk % Plan<true>::kTokAlign == 0,
+              "token chunk");
 
 enum Mode : int { kSwiGLU = 0, kGateDown = 1 };
 
@@ -161,6 +181,7 @@ struct TcParams {
   const uint8_t* s0_shared;
   const uint8_t* s1_shared;
   int sblocks_routed, sblocks_shared;
+  int chunk_rows;                // token rows of a unit at most (Plan::kChunk)
 };
 
 struct Unit {
@@ -183,7 +204,7 @@ MOE_DEV Unit decode_unit(const TcParams& p, int u) {
   // a group's rows split into nc chunks of (almost) equal size, so the
   // chunks that share a weight tile run at the same pace and keep reading
   // its lines from L2 together
-  const int nc = (rows + kMaxTok - 1) / kMaxTok;
+  const int nc = (rows + p.chunk_rows - 1) / p.chunk_rows;
   const int cs = (rows + nc - 1) / nc;
   Unit un;
   un.g = lo;
@@ -195,26 +216,34 @@ MOE_DEV Unit decode_unit(const TcParams& p, int u) {
   return un;
 }
 
-// Accumulator placement (identical in both CTAs). A unit of <= 128 tokens
-// takes one buffer (its two halves at columns base and base + 128); a larger
-// unit takes both buffers (halves at columns 0 and 256). The MMA issuer and
-// every epilogue thread replay the same sequence, so they agree on every
-// placement.
+// Accumulator placement over kCols columns (identical in both CTAs), by the
+// unit's MMA width n (its tokens rounded up to the N granule): a unit with
+// n <= kHalf (kCols / 4 rounded down to 32 columns) takes one of two
+// buffers, at 0 or kCols / 2 (its halves at base and base + kHalf), so the
+// next unit's MMAs overlap its epilogue; a wider unit takes both (halves at
+// 0 and kCols / 2). bf16 (512 columns): buffers for n <= 128; FP8 (320):
+// n <= 64. The MMA issuer and every epilogue thread replay the same
+// sequence, so they agree on every placement.
+template <uint32_t kCols>
 struct AccPlan {
+  static constexpr uint32_t kHalf = (kCols / 4) & ~31u;
   uint32_t next = 0;
-  MOE_DEV void place(int ntok, uint32_t& mask, uint32_t& base, uint32_t& stride) const {
-    if (ntok > kBufCols / 2) {
+  MOE_DEV void place(int n, uint32_t& mask, uint32_t& base, uint32_t& stride) const {
+    if (n > (int)kHalf) {
       mask = 3u;
       base = 0;
-      stride = kBufCols;
+      stride = kCols / 2;
     } else {
       mask = 1u << next;
-      base = next * kBufCols;
-      stride = kBufCols / 2;
+      base = next * (kCols / 2);
+      stride = kHalf;
     }
   }
-  MOE_DEV void advance(int ntok) { next = ntok > kBufCols / 2 ? 0u : next ^ 1u; }
+  MOE_DEV void advance(int n) { next = n > (int)kHalf ? 0u : next ^ 1u; }
 };
+// MMA width (N) of a unit of ntok tokens.
+template <bool FP8>
+MOE_DEV int mma_n(int ntok) { return (ntok + Plan<FP8>::kTokAlign - 1) & ~(Plan<FP8>::kTokAlign - 1); }
 
 struct Shared {
   uint64_t full[kSlots];       // CTA 0: stage bytes of both CTAs landed
@@ -236,12 +265,14 @@ static_assert(sizeof(Shared) <= 512, "barrier block");
 
 // The FP8 path's extra state (after Shared, inside the barrier block).
 struct SharedFp8 {
-  uint64_t conv_full[2];       // CTA 0: both CTAs' converters wrote the slot
-  uint64_t conv_empty[2];      // both: the pair MMAs finished reading the slot
+  uint64_t conv_full[kASlots];   // CTA 0: both CTAs' converters wrote the weight slot in TMEM (CTA 0's
+                                 // converters arrive, CTA 1's complete 4 transaction bytes)
+  uint64_t conv_empty[kASlots];  // both: the pair MMAs finished reading the slot
   int cvt_unit[2];             // the converter leader's unit for the converter warps
-  int cvt_info[2][3];          // its (g, f, tok0)
+  int cvt_info[2][2];          // its (g, f)
   int cvt_ok;                  // the leader's waits for the current stage succeeded
   uint32_t seen;               // stage fills this CTA's converters observed complete
+  uint32_t peer_word[kASlots];   // CTA 0: target of CTA 1's signalling stores (never read)
 };
 static_assert(512 + sizeof(SharedFp8) <= Plan<true>::kBarrierBytes, "FP8 barrier block");
 
@@ -252,22 +283,18 @@ MOE_DEV void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kWarps) : "m
 template <int kWarps>
 MOE_DEV void cvt_sync() { asm volatile("bar.sync 2, %0;" ::"n"(32 * kWarps) : "memory"); }
 
-// f16 pair -> the bf16 pair of its values times 2^-112, for f16 values
-// converted from e4m3: they carry 3 mantissa bits and are never f16
-// subnormals, so moving the f16 exponent field (5 bits) into the low bits of
-// the bf16 one and keeping the top 7 mantissa bits is exact and leaves each
-// value scaled by 2^(15 - 127). Zero stays zero.
-MOE_DEV uint32_t f16x2_to_bf16x2_scaled(uint32_t h) { return ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u); }
-
-// Four e4m3 codes (lowest byte first) -> two bf16 pairs (the values times
-// 2^-112); cvt.f16x2.e4m3x2 is exact.
-MOE_DEV void e4m3x4_to_bf16x4_scaled(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  uint32_t a, b;
-  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
-      : "=r"(a), "=r"(b)
-      : "r"(w));
-  lo = f16x2_to_bf16x2_scaled(a);
-  hi = f16x2_to_bf16x2_scaled(b);
+// Two e4m3 codes (bytes i and i + 1 of w, i = 0 or 2) -> the bf16 pair of
+// their values times 2^-120. For a code s eeee mmm the bf16 bit pattern
+// s 0000 eeee mmm 0000 has exponent field e and mantissa m / 8, i.e. the
+// value 2^(e - 127) (1 + m / 8) for e > 0 and the bf16 subnormal 2^-126 m / 8
+// for e = 0 (e4m3: 2^(e - 7) (1 + m / 8) and 2^-6 m / 8), and zero stays zero.
+// One byte permute spreads the two codes into 16-bit lanes with the sign
+// replicated into each high byte; a shift and a mask place the fields.
+template <int kSel>
+MOE_DEV uint32_t e4m3x2_to_bf16x2_scaled(uint32_t w) {
+  uint32_t t;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(t) : "r"(w), "n"(kSel));
+  return (t << 4) & 0x87F087F0u;
 }
 
 MOE_DEV uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
@@ -283,18 +310,19 @@ MOE_DEV uint32_t bf16x2_pow2(int e) {
 }
 
 // 16 e4m3 codes -> 16 bf16 values, each code value times 2^(sb - 127):
-// multiplied by 2^(112 + sb - 127) in one or (for sb > 142) two exact steps.
+// the values times 2^-120, multiplied by 2^(sb - 7) in one or (for
+// sb - 7 > 127) two exact steps (a power of two times a bf16 with 4
+// significant bits, subnormal or not, lands on a normal bf16).
 MOE_DEV void dequant16(const uint4 w, int sb, uint32_t (&o)[8]) {
-  const int e = sb - 15;                    // exponent of the total factor
+  const int e = sb - 7;                     // exponent of the total factor (>= -7)
   const int e1 = e > 127 ? 127 : e;
   const uint32_t f1 = bf16x2_pow2(e1);
   const uint32_t words[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    uint32_t lo, hi;
-    e4m3x4_to_bf16x4_scaled(words[i], lo, hi);
-    o[2 * i] = mul_bf16x2(lo, f1);
-    o[2 * i + 1] = mul_bf16x2(hi, f1);
+    // bytes [b0, sign b0, b1, sign b1] and [b2, sign b2, b3, sign b3]
+    o[2 * i] = mul_bf16x2(e4m3x2_to_bf16x2_scaled<0x9180>(words[i]), f1);
+    o[2 * i + 1] = mul_bf16x2(e4m3x2_to_bf16x2_scaled<0xB3A2>(words[i]), f1);
   }
   if (e > 127) {
     const uint32_t f2 = bf16x2_pow2(e - 127);
@@ -327,8 +355,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
   constexpr int kEpiWarps = PL::kEpiWarps, kCvtWarps = PL::kCvtWarps, kTBytes = tile_bytes<FP8>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* conv = smem + kRingBytes;  // FP8: the dequantised weight slots
-  float* tiles = reinterpret_cast<float*>(conv + PL::kConvBytes);
+  float* tiles = reinterpret_cast<float*>(smem + kRingBytes);
   Shared& sh = *reinterpret_cast<Shared*>(reinterpret_cast<uint8_t*>(tiles) + kTBytes);
   SharedFp8& shf = *reinterpret_cast<SharedFp8*>(reinterpret_cast<uint8_t*>(&sh) + 512);
 
@@ -363,8 +390,8 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
     sh.abort_flag = 0;
     sh.consumed = 0;
     if (FP8) {
-      for (int c = 0; c < PL::kConv; ++c) {
-        mbar_init(&shf.conv_full[c], 2);
+      for (int c = 0; c < kASlots; ++c) {
+        mbar_init(&shf.conv_full[c], 1);
         mbar_init(&shf.conv_empty[c], 1);
       }
       shf.seen = 0;
@@ -469,7 +496,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         const bool shared = un.g == p.N;
         const int K = shared ? p.k_shared : p.k_routed;
         const int nk = (K + kBK - 1) / kBK;
-        const int half_n = ((un.ntok + 15) & ~15) / 2;  // token rows per CTA
+        const int half_n = mma_n<FP8>(un.ntok) / 2;  // token rows per CTA
         // one token box per stage, the smallest of 32 / 64 / 128 rows that
         // covers this CTA's rows (the TMA engine's cost is per box, so a
         // single box beats several small ones even with rows to spare)
@@ -522,7 +549,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
     if (lane == 0 && first) {
       uint32_t consumed = 0;
       uint32_t uses[2] = {0u, 0u};
-      AccPlan plan;
+      AccPlan<PL::kAccCols> plan;
       bool ok = true;
       for (int i = 0; ok; ++i) {
         const int q = i % kRing;
@@ -536,10 +563,11 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         const Unit un = decode_unit(p, u);
         const int K = un.g == p.N ? p.k_shared : p.k_routed;
         const int nk = (K + kBK - 1) / kBK;
-        const uint32_t idesc = idesc_bf16_f32(256, (uint32_t)((un.ntok + 15) & ~15));
+        const int n = mma_n<FP8>(un.ntok);
+        const uint32_t idesc = idesc_bf16_f32(256, (uint32_t)n);
         uint32_t mask, base, stride;
-        plan.place(un.ntok, mask, base, stride);
-        plan.advance(un.ntok);
+        plan.place(n, mask, base, stride);
+        plan.advance(n);
         for (int b = 0; b < 2 && ok; ++b)
           if ((mask >> b) & 1u) {
             ok = mbar_wait_cluster_bounded(&sh.acc_empty[b], (uses[b] & 1u) ^ 1u, abort_flag);
@@ -552,8 +580,8 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
           const uint32_t s = consumed % kSlots, ph = (consumed / kSlots) & 1u;
           // FP8: the converted slot of this fill (both CTAs' converters have
           // observed its bytes land before they released it)
-          const uint32_t c = FP8 ? consumed % PL::kConv : 0u;
-          const bool landed = FP8 ? mbar_wait_cluster_bounded(&shf.conv_full[c], (consumed / PL::kConv) & 1u, abort_flag)
+          const uint32_t c = FP8 ? consumed % kASlots : 0u;
+          const bool landed = FP8 ? mbar_wait_cluster_bounded(&shf.conv_full[c], (consumed / kASlots) & 1u, abort_flag)
                                   : mbar_wait_cluster_bounded(&sh.full[s], ph, abort_flag);
           if (!landed) {
             ok = false;
@@ -562,13 +590,23 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
           ++consumed;
           tc_fence_after();
           const uint32_t stage_addr = smem_u32(smem + *reinterpret_cast<volatile uint32_t*>(&sh.slot_off[s]));
-          const uint32_t a_addr = FP8 ? smem_u32(conv + c * kATileBytes) : stage_addr;
-          const uint32_t b_addr = stage_addr + PL::kABytes;
+          const uint32_t b_addr = stage_addr + PL::kABytes;  // the token box follows the weights
+          if (FP8) {
+            // A: the converted slot in tensor memory, 8 columns per 16 K
+            const uint32_t a_t = tmem_base + PL::kAccCols + c * kASlotCols;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32);
-            umma_bf16_pair(d0, smem_desc_sw128(a_addr + kk * 32), bdesc, idesc, (kc | kk) != 0);
-            umma_bf16_pair(d1, smem_desc_sw128(a_addr + kHalfBytes + kk * 32), bdesc, idesc, (kc | kk) != 0);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32);
+              umma_bf16_pair_ts(d0, a_t + kk * 8, bdesc, idesc, (kc | kk) != 0);
+              umma_bf16_pair_ts(d1, a_t + kBK / 2 + kk * 8, bdesc, idesc, (kc | kk) != 0);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32);
+              umma_bf16_pair(d0, smem_desc_sw128(stage_addr + kk * 32), bdesc, idesc, (kc | kk) != 0);
+              umma_bf16_pair(d1, smem_desc_sw128(stage_addr + kHalfBytes + kk * 32), bdesc, idesc, (kc | kk) != 0);
+            }
           }
           umma_commit_pair_both(smem_u32(&sh.empty[s]));
           if (FP8) umma_commit_pair_both(smem_u32(&shf.conv_empty[c]));
@@ -601,7 +639,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
     __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(tiles) + ew * kTileBytes);
     const bool leader = threadIdx.x == 64;
     uint32_t uses[2] = {0u, 0u};
-    AccPlan plan;
+    AccPlan<PL::kAccCols> plan;
     for (int i = 0;; ++i) {
       // the leader takes the next unit and waits for its accumulator(s); the
       // epilogue warps then agree on the outcome and all run the unit or all leave
@@ -620,7 +658,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
             sh.epi_info[i & 1][3] = un.ntok;
             sh.epi_info[i & 1][4] = un.g == p.N ? un.tok0 : __ldg(p.grp_row0 + un.g) + un.tok0;
             uint32_t mask, base, stride;
-            plan.place(un.ntok, mask, base, stride);
+            plan.place(mma_n<FP8>(un.ntok), mask, base, stride);
             bool ok = true;
             for (int b = 0; b < 2 && ok; ++b)
               if ((mask >> b) & 1u) ok = mbar_wait_cluster_bounded(&sh.acc_full[b], uses[b] & 1u, abort_flag);
@@ -642,8 +680,8 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
       un.tok0 = load_volatile(&sh.epi_info[i & 1][2]);
       un.ntok = load_volatile(&sh.epi_info[i & 1][3]);
       uint32_t mask, base, stride;
-      plan.place(un.ntok, mask, base, stride);
-      plan.advance(un.ntok);
+      plan.place(mma_n<FP8>(un.ntok), mask, base, stride);
+      plan.advance(mma_n<FP8>(un.ntok));
       uses[0] += mask & 1u;
       uses[1] += (mask >> 1) & 1u;
       tc_fence_after();
@@ -752,13 +790,17 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
     }
   } else if (FP8) {
     // ----------------------------------------- FP8 converters (kCvtWarps) --
-    // Per fill, in the producer's order: wait for this CTA's bytes and for a
-    // free conversion slot, write the 256 x 64 dequantised bf16 weights in the
-    // 128-byte-swizzled layout the MMA descriptors expect (the layout a bf16
-    // TMA load would have produced), then tell the MMA issuer. A leader does
-    // the waits and the other warps follow its decision.
-    const int ct = threadIdx.x - 32 * (2 + kEpiWarps);  // 0 .. 32 kCvtWarps - 1
-    const bool cleader = ct == 0;
+    // Warp cw writes weight half cw / 4 of the rows in its TMEM lane quadrant:
+    // per fill, in the producer's order, it waits (through a leader) for this
+    // CTA's bytes and for a free weight slot, then each thread dequantises its
+    // row's 64 codes (the 64-byte-swizzled box row: chunk c at c ^ (row / 2 % 4))
+    // exactly into 32 columns of bf16 pairs, stores them to its TMEM lane and
+    // the leader tells the MMA issuer once every converter's stores are done.
+    const int cw = warp - (2 + kEpiWarps);   // 0 .. kCvtWarps - 1
+    const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+    const int hsel = cw >> 2;                // weight half
+    const int row = hsel * 128 + 32 * q + lane;  // row of the stage's code tile
+    const bool cleader = cw == 0 && lane == 0;
     uint32_t j = 0;  // fills converted
     bool alive = true;
     for (int i = 0; alive; ++i) {
@@ -791,23 +833,20 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
       const int nkb = K / kFp8Block;          // <= 64
       const int rowA = (shared ? 0 : g * p.a_rows_per_expert) + f * p.tile_cols + rank_rows;
       const int sblocks = shared ? p.sblocks_shared : p.sblocks_routed;
-      // this CTA's two 128-row halves: SwiGLU W1 / W3 rows of the same block,
-      // down GEMM two consecutive W2 blocks (a block past the matrix, whose
-      // rows load as zeros, takes the last block's scales)
-      const int rb0 = min(rowA / kFp8Block, sblocks - 1);
-      const int rb1 = MODE == kSwiGLU ? rb0 : min(rowA / kFp8Block + 1, sblocks - 1);
-      const uint8_t* sc0 = (shared ? p.s0_shared : p.s0_routed) + (int64_t)rb0 * nkb;
-      const uint8_t* sc1 = (MODE == kSwiGLU ? (shared ? p.s1_shared : p.s1_routed) : (shared ? p.s0_shared : p.s0_routed)) +
-                           (int64_t)rb1 * nkb;
-      // lane l holds the scale bytes of K blocks l and l + 32 of both halves
-      const int l = ct & 31;
-      const int sA0 = l < nkb ? __ldg(sc0 + l) : 0, sA1 = l + 32 < nkb ? __ldg(sc0 + l + 32) : 0;
-      const int sB0 = l < nkb ? __ldg(sc1 + l) : 0, sB1 = l + 32 < nkb ? __ldg(sc1 + l + 32) : 0;
+      // this warp's 128-row block: SwiGLU W1 (half 0) or W3 (half 1) rows of
+      // the same block; down GEMM two consecutive W2 blocks (a block past the
+      // matrix, whose rows load as zeros, takes the last block's scales)
+      const int rb = min(rowA / kFp8Block + (MODE == kSwiGLU ? 0 : hsel), sblocks - 1);
+      const uint8_t* sc = (MODE == kSwiGLU && hsel ? (shared ? p.s1_shared : p.s1_routed)
+                                                   : (shared ? p.s0_shared : p.s0_routed)) +
+                          (int64_t)rb * nkb;
+      // lane l holds the scale bytes of K blocks l and l + 32
+      const int sL = lane < nkb ? __ldg(sc + lane) : 0, sH = lane + 32 < nkb ? __ldg(sc + lane + 32) : 0;
       for (int kc = 0; kc < nk; ++kc, ++j) {
-        const uint32_t s = j % kSlots, c = j % PL::kConv;
+        const uint32_t s = j % kSlots, c = j % kASlots;
         if (cleader) {
           const bool ok = mbar_wait_bounded(&sh.full[s], (j / kSlots) & 1u, abort_flag) &&
-                          mbar_wait_cluster_bounded(&shf.conv_empty[c], ((j / PL::kConv) & 1u) ^ 1u, abort_flag);
+                          mbar_wait_cluster_bounded(&shf.conv_empty[c], ((j / kASlots) & 1u) ^ 1u, abort_flag);
           if (ok) shf.seen = j + 1;
           else {
             *abort_flag = 1;
@@ -820,34 +859,31 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
           alive = false;
           break;
         }
+        tc_fence_after();  // the MMAs that read this slot before have completed
         const int kb = kc >> 1;  // 64-wide K block -> 128-wide scale block
-        const int sb0 = __shfl_sync(0xffffffffu, kb < 32 ? sA0 : sA1, kb & 31);
-        const int sb1 = __shfl_sync(0xffffffffu, kb < 32 ? sB0 : sB1, kb & 31);
+        const int sb = __shfl_sync(0xffffffffu, kb < 32 ? sL : sH, kb & 31);
         const uint32_t raw = smem_u32(smem) + *reinterpret_cast<volatile uint32_t*>(&sh.slot_off[s]);
-        const uint32_t dst = smem_u32(conv) + c * kATileBytes;
-        constexpr int kPieces = kA8Bytes / 16 / (32 * kCvtWarps);  // 16-byte pieces per thread
-        uint4 wv[kPieces];  // all loads first: independent work for the conversion below
+        const uint32_t src = raw + row * kBK;
+        uint4 wv[4];
 #pragma unroll
-        for (int it = 0; it < kPieces; ++it) {
-          const int v = ct + 32 * kCvtWarps * it;  // 16-byte piece: row v / 4 (of 256), bytes 16 (v % 4) ..
-          wv[it] = ld_shared_v4(raw + (v >> 2) * kBK + (v & 3) * 16);
-        }
+        for (int c4 = 0; c4 < 4; ++c4) wv[c4] = ld_shared_v4(src + ((c4 ^ ((row >> 1) & 3)) << 4));
+        uint32_t o[32];
 #pragma unroll
-        for (int it = 0; it < kPieces; ++it) {
-          const int v = ct + 32 * kCvtWarps * it;
-          const int r = v >> 2, q4 = v & 3;
-          uint32_t o[8];
-          dequant16(wv[it], r < 128 ? sb0 : sb1, o);
-          const int rr = r & 127;
-          const uint32_t row = dst + (r >> 7) * kHalfBytes + rr * (kBK * 2);
-          st_shared_v4(row + (((2 * q4) ^ (rr & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
-          st_shared_v4(row + (((2 * q4 + 1) ^ (rr & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t v[8];
+          dequant16(wv[c4], sb, v);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[8 * c4 + e] = v[e];
         }
-        fence_proxy_async_smem();  // the tensor cores read the slot through the async proxy
+        tmem_st32(tmem_base + ((uint32_t)(32 * q) << 16) + PL::kAccCols + c * kASlotCols + hsel * (kBK / 2), o);
+        tmem_wait_st();
+        tc_fence_before();
         cvt_sync<kCvtWarps>();
         if (cleader) {
-          if (first) mbar_arrive(&shf.conv_full[c]);
-          else mbar_arrive_cluster(in_first(&shf.conv_full[c]));
+          // CTA 1 signals through an asynchronous store (a blocking
+          // cluster-scope arrive costs about 1000 cycles per stage)
+          if (first) mbar_arrive_expect_tx(&shf.conv_full[c], 4);
+          else st_async_u32(in_first(&shf.peer_word[c]), j, in_first(&shf.conv_full[c]));
         }
       }
     }
@@ -893,9 +929,10 @@ bool make_store_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
   return make_tmap_bf16_swz(m, base, rows, cols, 32, 32, 64);
 }
 
-// FP8 weight codes: 64 bytes x box_rows rows, unswizzled (the converters read them row by row).
+// FP8 weight codes: 64 bytes x box_rows rows, 64-byte swizzle (each
+// converter thread reads one row; a warp's 32 rows then cover all banks).
 bool make_tmap_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  return make_tmap_u8(m, base, rows, cols, kBK, box_rows);
+  return make_tmap_u8(m, base, rows, cols, kBK, box_rows, 64);
 }
 
 template <int MODE, bool FP8>
@@ -948,10 +985,10 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   const int sms = device_sm_count();
   cudaError_t err0 = cudaMemsetAsync(a.sched, 0, 2 * sizeof(int), s);
   if (err0 != cudaSuccess) return err0;
-  const int64_t chunks_bound =
-      (p.R + kMaxTok - 1) / kMaxTok + p.N + (p.ns > 0 ? (p.T + kMaxTok - 1) / kMaxTok : 0);
-
   const bool fp8 = a.fp8;
+  const int cm = fp8 ? Plan<true>::kChunk : Plan<false>::kChunk;  // token rows of a unit at most
+  const int64_t chunks_bound = (p.R + cm - 1) / cm + p.N + (p.ns > 0 ? (p.T + cm - 1) / cm : 0);
+
   // weight maps: bf16 tiles, or the FP8 codes (plus their block scales)
   auto wmap = [&](CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     return fp8 ? make_tmap_codes(m, base, rows, cols, box_rows) : make_tmap(m, base, rows, cols, box_rows);
@@ -990,6 +1027,7 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g1.s1_shared = a.Ws3s;
   g1.sblocks_routed = (int)((int64_t)p.N * p.F / kFp8Block);
   g1.sblocks_shared = p.nsF / kFp8Block;
+  g1.chunk_rows = cm;
   const int64_t max_cols1 = p.F > p.nsF ? p.F : p.nsF;
   const int64_t units1 = chunks_bound * ((max_cols1 + kTcBN1 - 1) / kTcBN1);
   const int grid1 = (int)(units1 < sms ? units1 : sms);
@@ -1027,6 +1065,7 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g2.s0_shared = a.Ws2s;
   g2.sblocks_routed = (int)((int64_t)p.N * p.d / kFp8Block);
   g2.sblocks_shared = p.d / kFp8Block;
+  g2.chunk_rows = cm;
   const int64_t units2 = chunks_bound * ((p.d + kTcBN2 - 1) / kTcBN2);
   const int grid2 = (int)(units2 < sms ? units2 : sms);
   // the down GEMM overlaps the SwiGLU GEMM's drain unless an event must be

@@ -15,8 +15,11 @@ namespace moe {
 // covers at most kTcBM token rows of one group (UMMA N) and kTcBN1 SwiGLU
 // features (two pair UMMAs of M = 256: W1 rows and the same W3 rows) or
 // kTcBN2 model columns of the down projection (two pair UMMAs of M = 256).
+// With FP8 weights a unit covers at most kTcBM8 token rows: its bf16 weight
+// tiles live in tensor memory beside the accumulators.
 // The fp32 SIMT GEMMs use 64 x 64 tiles.
 constexpr int kTcBM = 256;
+constexpr int kTcBM8 = 160;
 constexpr int kTcBN1 = 256;
 constexpr int kTcBN2 = 512;
 constexpr int kSimtBM = 64;
@@ -72,9 +75,10 @@ struct DispatchBuffers {
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                     uint32_t box_rows, bool swizzle128);
 // uint8 row-major [rows, cols] (FP8 codes) with a box of box_cols bytes x
-// box_rows rows, no swizzle, 256-byte L2 promotion; zero fill outside.
+// box_rows rows, 256-byte L2 promotion, zero fill outside; swizzle_bytes 64
+// gives the 64-byte swizzle (box_cols must then be 64), 0 none.
 bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                  uint32_t box_rows);
+                  uint32_t box_rows, int swizzle_bytes = 0);
 // The same with a swizzle of 0, 64 or 128 bytes.
 bool make_tmap_bf16_swz(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                         uint32_t box_rows, int swizzle_bytes);

@@ -186,7 +186,8 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
   if ((e0 = mark_stage(1, s)) != cudaSuccess) return cuda_fail(e0);
   const bool tc = p.dtype == MOE_BF16;
   DispatchBuffers db = dispatch_buffers(L, ws, idx, gates);
-  cudaError_t e = launch_dispatch(p, db, tc ? kTcBM : kSimtBM, tc ? kTcBN1 : kSimtBN,
+  // unit tables for the GEMMs: FP8 weights cut groups into chunks of at most kTcBM8 rows
+  cudaError_t e = launch_dispatch(p, db, tc ? (fp8 ? kTcBM8 : kTcBM) : kSimtBM, tc ? kTcBN1 : kSimtBN,
                                   tc ? kTcBN2 : kSimtBN, s);
   if (e == cudaSuccess) e = mark_stage(2, s);
   if (e != cudaSuccess) return cuda_fail(e);
