@@ -249,9 +249,11 @@ struct Shared {
   uint64_t full[kSlots];       // CTA 0: stage bytes of both CTAs landed
   uint64_t empty[kSlots];      // both: the pair MMAs finished reading the stage
   uint64_t acc_full[2];        // both: accumulator buffer complete
-  uint64_t acc_empty[2];       // CTA 0: both CTAs' epilogues released the buffer
+  uint64_t acc_empty[2];       // CTA 0: both CTAs' epilogues released the buffer (CTA 0's epilogue
+                               // warps arrive, CTA 1's complete 4 transaction bytes each)
   uint64_t ring_full[kRing];   // both: unit id published
-  uint64_t ring_empty[kRing];  // CTA 0: every reader of the pair took the id
+  uint64_t ring_empty[kRing];  // CTA 0: every reader of the pair took the id (CTA 0's readers
+                               // arrive, CTA 1's complete 4 transaction bytes each)
   uint64_t drained;            // both: all pair MMAs completed
   uint32_t slot_off[kSlots];   // byte offset of each stage in the ring
   int ring[kRing];
@@ -260,6 +262,7 @@ struct Shared {
   uint32_t tmem_base;
   int abort_flag;
   uint32_t consumed;           // stage fills the MMA issuer observed complete
+  uint32_t sink;               // CTA 0: target of CTA 1's signalling stores (never read)
 };
 static_assert(sizeof(Shared) <= 512, "barrier block");
 
@@ -370,6 +373,12 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
   // contiguous 256-row box whose first and second 128 rows are halves 0 and
   // 1; so TMEM lane l of half h in CTA r is output column 256 r + 128 h + l.
   const int rank_rows = (MODE == kSwiGLU ? 128 : 256) * (int)rank;
+  // Readers of each unit id in each CTA (producer or MMA issuer, epilogue
+  // leader, FP8 converter leader). The pair's cross-CTA signals are
+  // asynchronous stores that complete transaction bytes on the other CTA's
+  // barrier (st.async): a blocking cluster-scope mbarrier arrive costs the
+  // signalling thread about 1000 cycles.
+  constexpr int kRingReaders = FP8 ? 3 : 2;
   const int half_cols = MODE == kSwiGLU ? 0 : 128;
 
   if (threadIdx.x == 0) {
@@ -379,12 +388,12 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.acc_full[b], 1);
-      mbar_init(&sh.acc_empty[b], 2 * kEpiWarps);
+      mbar_init(&sh.acc_empty[b], kEpiWarps);
     }
     for (int q = 0; q < kRing; ++q) {
       mbar_init(&sh.ring_full[q], 1);
-      // both CTAs: producer or MMA issuer, epilogue leader (and FP8 converter leader)
-      mbar_init(&sh.ring_empty[q], FP8 ? 6 : 4);
+      // CTA 0's readers: MMA issuer, epilogue leader (and FP8 converter leader)
+      mbar_init(&sh.ring_empty[q], kRingReaders);
     }
     mbar_init(&sh.drained, 1);
     sh.abort_flag = 0;
@@ -475,16 +484,18 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
           u = atomicAdd(p.sched, 1);
           if (u >= total_units) u = -1;
           sh.ring[q] = u;
-          st_cluster_u32(peer(&sh.ring[q]), (uint32_t)u);
           mbar_arrive(&sh.ring_full[q]);
-          mbar_arrive_cluster(peer(&sh.ring_full[q]));
+          // the id itself is the 4 transaction bytes of the peer's ring_full
+          st_async_u32(peer(&sh.ring[q]), (uint32_t)u, peer(&sh.ring_full[q]));
         } else {
+          // this CTA's ring_full phase: one arrival (here) and the 4 bytes of CTA 0's store
+          mbar_arrive_expect_tx(&sh.ring_full[q], 4);
           if (!mbar_wait_cluster_bounded(&sh.ring_full[q], (i / kRing) & 1, abort_flag)) {
             ok = false;
             break;
           }
           u = load_volatile(&sh.ring[q]);
-          mbar_arrive_cluster(in_first(&sh.ring_empty[q]));
+          st_async_u32(in_first(&sh.sink), 0u, in_first(&sh.ring_empty[q]));
         }
         if (u < 0) {
           // no units left for this CTA: the down GEMM may start on SMs as
@@ -558,7 +569,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
           break;
         }
         const int u = load_volatile(&sh.ring[q]);
-        mbar_arrive(&sh.ring_empty[q]);
+        mbar_arrive_expect_tx(&sh.ring_empty[q], 4 * kRingReaders);  // and CTA 1's readers' stores
         if (u < 0) break;
         const Unit un = decode_unit(p, u);
         const int K = un.g == p.N ? p.k_shared : p.k_routed;
@@ -649,7 +660,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         if (mbar_wait_cluster_bounded(&sh.ring_full[qr], (i / kRing) & 1, abort_flag)) {
           u = load_volatile(&sh.ring[qr]);
           if (first) mbar_arrive(&sh.ring_empty[qr]);
-          else mbar_arrive_cluster(in_first(&sh.ring_empty[qr]));
+          else st_async_u32(in_first(&sh.sink), 0u, in_first(&sh.ring_empty[qr]));
           if (u >= 0) {
             const Unit un = decode_unit(p, u);
             sh.epi_info[i & 1][0] = un.g;
@@ -783,8 +794,9 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
       if (lane == 0) {
         for (int b = 0; b < 2; ++b)
           if ((mask >> b) & 1u) {
-            if (first) mbar_arrive(&sh.acc_empty[b]);
-            else mbar_arrive_cluster(in_first(&sh.acc_empty[b]));
+            if (!first) st_async_u32(in_first(&sh.sink), 0u, in_first(&sh.acc_empty[b]));
+            else if (ew == 0) mbar_arrive_expect_tx(&sh.acc_empty[b], 4 * kEpiWarps);  // and CTA 1's warps' stores
+            else mbar_arrive(&sh.acc_empty[b]);
           }
       }
     }
@@ -810,7 +822,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         if (mbar_wait_cluster_bounded(&sh.ring_full[qr], (i / kRing) & 1, abort_flag)) {
           u = load_volatile(&sh.ring[qr]);
           if (first) mbar_arrive(&sh.ring_empty[qr]);
-          else mbar_arrive_cluster(in_first(&sh.ring_empty[qr]));
+          else st_async_u32(in_first(&sh.sink), 0u, in_first(&sh.ring_empty[qr]));
           if (u >= 0) {
             const Unit un = decode_unit(p, u);
             shf.cvt_info[i & 1][0] = un.g;
