@@ -270,13 +270,14 @@ class Layer:
         import torch
         xh = self.x.cpu().pin_memory()
         yh = torch.empty_like(xh).pin_memory()
+        fwd = self.moe.forward_host_fp8 if self.s.wdtype == "fp8" else self.moe.forward_host
         for _ in range(warmup):
-            self.moe.forward_host(self.cfg, self.s.T, xh, *self.wargs, yh, self.ws, stream=self.stream)
+            fwd(self.cfg, self.s.T, xh, *self.wargs, yh, self.ws, stream=self.stream)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(self.stream)
         for _ in range(steps):
-            self.moe.forward_host(self.cfg, self.s.T, xh, *self.wargs, yh, self.ws, stream=self.stream)
+            fwd(self.cfg, self.s.T, xh, *self.wargs, yh, self.ws, stream=self.stream)
         e1.record(self.stream)
         torch.cuda.synchronize()
         self.moe.workspace_release(self.ws)
@@ -391,10 +392,12 @@ def run_ours(args, rank, world, local_rank):
                    "n_shared": s.n_shared, "d_ff": s.d_ff, "top_k": s.top_k, "global_batch": world * s.T,
                    "parallelism": f"dp{world} (independent replicas, no collective)",
                    "l2": "inputs larger than L2: every step streams "
-                         f"{(A['U'] + s.n_shared) * 3 * s.d * s.d_ff * 2 / 1e9:.1f} GB of expert weights"},
+                         f"{(A['U'] + s.n_shared) * 3 * s.d * s.d_ff * weight_bytes_per_element(s) / 1e9:.1f} "
+                         "GB of expert weights"},
         "e2e": {"value": round(world * s.T / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
-                "api": "moe_forward_host (pinned host x in, y out, every step)"},
+                "api": ("moe_forward_host_fp8" if s.wdtype == "fp8" else "moe_forward_host")
+                       + " (pinned host x in, y out, every step)"},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "roofline": {"bound": "hbm", "kernel": "expert_gemm_tc_kernel<SwiGLU>",
                      "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",

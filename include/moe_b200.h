@@ -192,7 +192,7 @@ typedef struct moe_fp8_matrix {
  * moe_forward with FP8 expert weights (routed and shared): the same layer,
  * tokens, router (W_r bf16), outputs and workspace as moe_forward with
  * cfg->dtype == MOE_BF16. Each weight tile is dequantised exactly to bf16 in
- * shared memory (a power-of-two scale times an e4m3 value is a bf16 value)
+ * tensor memory (a power-of-two scale times an e4m3 value is a bf16 value)
  * and multiplied on the tensor cores as in the bf16 path, so the result
  * equals moe_forward run on the dequantised weights (bit for bit, as long as
  * every dequantised weight is a normal bf16 number). Weight bytes streamed
@@ -240,6 +240,20 @@ MOE_API moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x
  * Errors: MOE_ERR_CUDA if the workspace's device cannot be made current.
  */
 MOE_API moe_status moe_workspace_release(const void* ws);
+
+/*
+ * moe_forward_host with FP8 expert weights: the x and y host buffers,
+ * staging, ordering and copy stream of moe_forward_host around the device
+ * forward of moe_forward_fp8 (same weights arguments, requirements and
+ * results). The workspace is sized by moe_workspace_size_host; the per-
+ * workspace state is shared with moe_forward_host and freed by
+ * moe_workspace_release.
+ */
+MOE_API moe_status moe_forward_host_fp8(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
+                                const float* b, const moe_fp8_matrix* W1, const moe_fp8_matrix* W3,
+                                const moe_fp8_matrix* W2, const moe_fp8_matrix* Ws1,
+                                const moe_fp8_matrix* Ws3, const moe_fp8_matrix* Ws2, void* y_host,
+                                void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Reads (and optionally clears) the device-status word of a workspace used

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ["moe_workspace_size", "moe_workspace_size_host", "moe_route", "moe_dispatch", "moe_forward",
            "moe_forward_fp8", "moe_dispatch_rows", "moe_experts_workspace_size", "moe_experts", "moe_combine",
            "moe_ep_reorder",
-           "moe_forward_host", "moe_workspace_release", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update", "moe_selftest_wait_timeout",
+           "moe_forward_host", "moe_forward_host_fp8", "moe_workspace_release", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update", "moe_selftest_wait_timeout",
            "moe_status_string", "moe_last_cuda_error"]
 STAGES = ["router", "dispatch", "gather", "gemm_swiglu", "gemm_gate", "combine"]
 
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
         FP8P = ctypes.POINTER(Fp8Matrix)
         L.moe_forward_fp8.argtypes = [CFG, I64, P, P, P, FP8P, FP8P, FP8P, FP8P, FP8P, FP8P, P, P, P, P, SZ, P]
         L.moe_forward_host.argtypes = [CFG, I64, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_forward_host_fp8.argtypes = [CFG, I64, P, P, P, FP8P, FP8P, FP8P, FP8P, FP8P, FP8P, P, P, SZ, P]
         L.moe_workspace_release.argtypes = [P]
         L.moe_device_status.argtypes = [CFG, I64, P, SZ, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32), P]
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
@@ -259,6 +260,16 @@ def forward_host(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, 
                                                       _ptr(W1), _ptr(W3), _ptr(W2), _ptr(Ws1), _ptr(Ws3),
                                                       _ptr(Ws2), _ptr(y_host), _ptr(ws), ws_bytes,
                                                       _stream(stream)))
+
+
+def forward_host_fp8(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, ws_bytes=None,
+                     stream=None):
+    """moe_forward_host with FP8 expert weights ((codes, scales) pairs as in forward_fp8)."""
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    _check("moe_forward_host_fp8", lib().moe_forward_host_fp8(ctypes.byref(cfg), T, _ptr(x_host), _ptr(W_r),
+                                                              _ptr(b), _fp8(W1), _fp8(W3), _fp8(W2), _fp8(Ws1),
+                                                              _fp8(Ws3), _fp8(Ws2), _ptr(y_host), _ptr(ws),
+                                                              ws_bytes, _stream(stream)))
 
 
 def workspace_release(ws) -> None:

@@ -401,6 +401,79 @@ __global__ void check_counts_kernel(const int32_t* __restrict__ counts, int E, i
 }
 
 }  // namespace
+// Configuration checks of the FP8 entry points.
+moe_status check_fp8_cfg(const Problem& p) {
+  if (p.dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  constexpr int kBlock = 128, kMaxK = 8192;  // block size; K / 128 scale blocks per lane pair
+  if (p.d % kBlock || p.F % kBlock || p.nsF % kBlock || p.d > kMaxK || p.F > kMaxK || p.nsF > kMaxK)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// Pointer checks of the FP8 entry points (codes of W1..Ws2 in m; the shared
+// ones may be NULL iff n_shared == 0); fills the scale pointers.
+moe_status check_fp8_ptrs(const Problem& p, const void* W_r, const float* b, const moe_fp8_matrix* const (&m)[6],
+                          Fp8Scales* sc) {
+  if (!W_r || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
+  if (b && (reinterpret_cast<uintptr_t>(b) & 3u)) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i) {
+    const bool need = i < 3 || p.ns > 0;
+    sc->s[i] = nullptr;
+    if (!need) continue;
+    if (!m[i] || !m[i]->codes || !m[i]->scales || !aligned16(m[i]->codes)) return MOE_ERR_INVALID_ARG;
+    sc->s[i] = m[i]->scales;
+  }
+  return MOE_OK;
+}
+
+const void* fp8_codes(const Problem& p, const moe_fp8_matrix* const (&m)[6], int i) {
+  return (i < 3 || p.ns > 0) ? m[i]->codes : nullptr;
+}
+
+// The host-buffer pipeline of moe_forward_host(_fp8) around one device
+// forward, run(x_device, y_device) on stream s: x is copied into one of the
+// workspace's two staging slots on the workspace's copy stream (overlapping
+// the previous call), y is copied back to the host on s.
+template <class Run>
+moe_status forward_host_pipe(const Problem& p, const Layout& L, const void* x_host, void* y_host, void* ws,
+                             cudaStream_t s, Run run) {
+  const size_t bytes = (size_t)p.T * p.d * p.elem;
+  void* yd = at<void>(ws, L.y_stage);
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* hp = nullptr;
+  cudaError_t e = host_pipe_locked(ws, &hp);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const size_t key[3] = {L.x_stage[0], L.x_stage[1], bytes};
+  if (std::memcmp(key, hp->stage_key, sizeof(key)) != 0) hp->relayout = true;
+  if (hp->relayout) {
+    // another layout (or device work) since the last host call: the copy may
+    // land on regions the previous call still uses, so wait for all of it
+    hp->slot_used[0] = hp->slot_used[1] = false;
+    if (hp->done_recorded) e = cudaStreamWaitEvent(hp->copy, hp->done, 0);
+    hp->calls = 0;
+  }
+  const int slot = (int)(hp->calls & 1u);
+  void* xd = at<void>(ws, L.x_stage[slot]);
+  if (e == cudaSuccess && hp->slot_used[slot]) e = cudaStreamWaitEvent(hp->copy, hp->x_free[slot], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, hp->copy);
+  if (e == cudaSuccess) e = cudaEventRecord(hp->x_ready, hp->copy);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->x_ready, 0);
+  if (e != cudaSuccess) return cuda_fail(e);
+  moe_status st = run(xd, yd);
+  if (st != MOE_OK) return st;
+  // the slot is free again once this call's kernels are done
+  if ((e = cudaEventRecord(hp->x_free[slot], s)) != cudaSuccess) return cuda_fail(e);
+  hp->slot_used[slot] = true;
+  e = cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaEventRecord(hp->done, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  hp->done_recorded = true;
+  hp->relayout = false;
+  std::memcpy(hp->stage_key, key, sizeof(key));
+  ++hp->calls;
+  return MOE_OK;
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -496,26 +569,17 @@ moe_status moe_forward_fp8(const moe_cfg* cfg, int64_t T, const void* x, const v
   Problem p;
   moe_status st = make_problem(cfg, T, &p);
   if (st != MOE_OK) return st;
-  if (p.dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
-  constexpr int kBlock = 128, kMaxK = 8192;  // block size; K / 128 scale blocks per lane pair
-  if (p.d % kBlock || p.F % kBlock || p.nsF % kBlock || p.d > kMaxK || p.F > kMaxK || p.nsF > kMaxK)
-    return MOE_ERR_UNSUPPORTED;
+  if ((st = check_fp8_cfg(p)) != MOE_OK) return st;
   if (T == 0) return MOE_OK;
-  if (!x || !y || !aligned16(x) || !aligned16(y) || !W_r || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
-  if (b && (reinterpret_cast<uintptr_t>(b) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   const moe_fp8_matrix* m[6] = {W1, W3, W2, Ws1, Ws3, Ws2};
-  for (int i = 0; i < 6; ++i) {
-    const bool need = i < 3 || p.ns > 0;
-    if (!need) continue;
-    if (!m[i] || !m[i]->codes || !m[i]->scales || !aligned16(m[i]->codes)) return MOE_ERR_INVALID_ARG;
-  }
+  Fp8Scales sc{};
+  if ((st = check_fp8_ptrs(p, W_r, b, m, &sc)) != MOE_OK) return st;
   Layout L = make_layout(p);
   if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
-  Fp8Scales sc{};
-  for (int i = 0; i < 6; ++i) sc.s[i] = (i < 3 || p.ns > 0) ? m[i]->scales : nullptr;
-  auto codes = [&](int i) -> const void* { return (i < 3 || p.ns > 0) ? m[i]->codes : nullptr; };
-  st = forward_device(p, L, x, W_r, b, codes(0), codes(1), codes(2), codes(3), codes(4), codes(5), y, topk_idx_out,
-                      gates_out, ws, (cudaStream_t)stream, &sc);
+  st = forward_device(p, L, x, W_r, b, fp8_codes(p, m, 0), fp8_codes(p, m, 1), fp8_codes(p, m, 2),
+                      fp8_codes(p, m, 3), fp8_codes(p, m, 4), fp8_codes(p, m, 5), y, topk_idx_out, gates_out, ws,
+                      (cudaStream_t)stream, &sc);
   if (st != MOE_OK) return st;
   cudaError_t e = note_device_use(ws, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
@@ -534,41 +598,33 @@ moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, c
   Layout L = make_layout(p);
   if ((st = check_ws(L, ws, ws_bytes, L.total_host)) != MOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  const size_t bytes = (size_t)p.T * p.d * p.elem;
-  void* yd = at<void>(ws, L.y_stage);
-  std::lock_guard<std::mutex> lock(g_pipe_mu);
-  HostPipe* hp = nullptr;
-  cudaError_t e = host_pipe_locked(ws, &hp);
-  if (e != cudaSuccess) return cuda_fail(e);
-  const size_t key[3] = {L.x_stage[0], L.x_stage[1], bytes};
-  if (std::memcmp(key, hp->stage_key, sizeof(key)) != 0) hp->relayout = true;
-  if (hp->relayout) {
-    // another layout (or device work) since the last host call: the copy may
-    // land on regions the previous call still uses, so wait for all of it
-    hp->slot_used[0] = hp->slot_used[1] = false;
-    if (hp->done_recorded) e = cudaStreamWaitEvent(hp->copy, hp->done, 0);
-    hp->calls = 0;
-  }
-  const int slot = (int)(hp->calls & 1u);
-  void* xd = at<void>(ws, L.x_stage[slot]);
-  if (e == cudaSuccess && hp->slot_used[slot]) e = cudaStreamWaitEvent(hp->copy, hp->x_free[slot], 0);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, hp->copy);
-  if (e == cudaSuccess) e = cudaEventRecord(hp->x_ready, hp->copy);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->x_ready, 0);
-  if (e != cudaSuccess) return cuda_fail(e);
-  st = forward_device(p, L, xd, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, yd, nullptr, nullptr, ws, s);
+  return forward_host_pipe(p, L, x_host, y_host, ws, s, [&](const void* xd, void* yd) {
+    return forward_device(p, L, xd, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, yd, nullptr, nullptr, ws, s);
+  });
+}
+
+moe_status moe_forward_host_fp8(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
+                                const float* b, const moe_fp8_matrix* W1, const moe_fp8_matrix* W3,
+                                const moe_fp8_matrix* W2, const moe_fp8_matrix* Ws1, const moe_fp8_matrix* Ws3,
+                                const moe_fp8_matrix* Ws2, void* y_host, void* ws, size_t ws_bytes,
+                                void* stream) {
+  Problem p;
+  moe_status st = make_problem(cfg, T, &p);
   if (st != MOE_OK) return st;
-  // the slot is free again once this call's kernels are done
-  if ((e = cudaEventRecord(hp->x_free[slot], s)) != cudaSuccess) return cuda_fail(e);
-  hp->slot_used[slot] = true;
-  e = cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaEventRecord(hp->done, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  hp->done_recorded = true;
-  hp->relayout = false;
-  std::memcpy(hp->stage_key, key, sizeof(key));
-  ++hp->calls;
-  return MOE_OK;
+  if ((st = check_fp8_cfg(p)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
+  const moe_fp8_matrix* m[6] = {W1, W3, W2, Ws1, Ws3, Ws2};
+  Fp8Scales sc{};
+  if ((st = check_fp8_ptrs(p, W_r, b, m, &sc)) != MOE_OK) return st;
+  Layout L = make_layout(p);
+  if ((st = check_ws(L, ws, ws_bytes, L.total_host)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  return forward_host_pipe(p, L, x_host, y_host, ws, s, [&](const void* xd, void* yd) {
+    return forward_device(p, L, xd, W_r, b, fp8_codes(p, m, 0), fp8_codes(p, m, 1), fp8_codes(p, m, 2),
+                          fp8_codes(p, m, 3), fp8_codes(p, m, 4), fp8_codes(p, m, 5), yd, nullptr, nullptr, ws, s,
+                          &sc);
+  });
 }
 
 moe_status moe_workspace_release(const void* ws) {

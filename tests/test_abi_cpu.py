@@ -43,6 +43,13 @@ def test_library_exports_every_header_function(L):
     assert {s for s in syms if s.startswith("moe_")} == set(header_functions())
 
 
+def test_binding_declares_argument_types(L):
+    """Every function the binding calls has ctypes argument types: without
+    them a 64-bit argument (T, a byte count) is passed as a 32-bit int."""
+    for name in moe.EXPORTS:
+        assert getattr(L, name).argtypes is not None, name
+
+
 def test_cfg_struct_matches_header():
     src = open(HEADER).read()
     body = re.search(r"typedef struct moe_cfg \{(.*?)\} moe_cfg;", src, flags=re.S).group(1)

@@ -149,3 +149,31 @@ def test_fp8_rejects_unsupported_shapes():
         moe.forward_fp8(cfg32, 4, 16, 16, None, (16, 16), (16, 16), (16, 16), None, None, None, 16, 256,
                         ws_bytes=0)
     assert ei.value.status == 1
+
+
+def test_fp8_host_entry_matches_device_entry():
+    """moe_forward_host_fp8 (pinned host x in, y out) gives moe_forward_fp8's
+    bits, on back-to-back calls that alternate the two staging slots and on a
+    smaller batch on the same workspace afterwards."""
+    s = SMALL["fp8_ragged"]
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    cfg = cfg_of(s)
+    wargs = (w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"])
+    y_dev, _, _ = run_fp8(s, w, x)
+    ws = workspace(cfg, s.T, host=True)
+    xh = x.cpu().pin_memory()
+    yh = [torch.empty_like(xh).pin_memory() for _ in range(3)]
+    for i in range(3):
+        moe.forward_host_fp8(cfg, s.T, xh, *wargs, yh[i], ws)
+    torch.cuda.synchronize()
+    for i in range(3):
+        assert torch.equal(yh[i], y_dev.cpu())
+    T2 = 200
+    y2_dev, _, _ = run_fp8(s, w, x[:T2].contiguous())
+    y2h = torch.empty((T2, s.d), dtype=xh.dtype).pin_memory()
+    moe.forward_host_fp8(cfg, T2, xh[:T2].contiguous().pin_memory(), *wargs, y2h, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y2h, y2_dev.cpu())
+    assert moe.device_status(cfg, T2, ws) == 0
+    moe.workspace_release(ws)
