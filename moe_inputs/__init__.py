@@ -117,6 +117,8 @@ SHAPES["v2_device_limited_bf16"] = SHAPES["v2_layer_bf16"].with_(name="v2_device
 # scale per 128 x 128 block); tokens, router and bias as in the bf16 layer.
 SHAPES["v3_prefill_fp8"] = SHAPES["v3_prefill_bf16"].with_(name="v3_prefill_fp8", wdtype="fp8")
 SHAPES["v3_decode_fp8"] = SHAPES["v3_decode_bf16"].with_(name="v3_decode_fp8", wdtype="fp8")
+# The small profiling layer with FP8 weights (1.5 GB of codes: ncu full-section captures)
+SHAPES["v3_profile_32e_fp8"] = SHAPES["v3_profile_32e"].with_(name="v3_profile_32e_fp8", wdtype="fp8")
 ORDER = ["gshard_tiny_f32", "dsmoe_2b_bf16", "v2_layer_bf16", "v3_prefill_bf16", "v3_decode_bf16"]
 
 
