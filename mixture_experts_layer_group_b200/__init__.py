@@ -307,7 +307,10 @@ class MoELayer:
     """A DeepSeekMoE layer bound to device-resident weights and a workspace.
 
     weights: dict with W_r, b (or None), W1, W3, W2 and, when n_shared > 0,
-    Ws1, Ws3, Ws2 -- torch CUDA tensors in the layouts of the C ABI.
+    Ws1, Ws3, Ws2 -- torch CUDA tensors in the layouts of the C ABI. Expert
+    weights given as (codes, scales) pairs of uint8 tensors are FP8 (e4m3 with
+    a power-of-two scale per 128 x 128 block) and run through
+    moe_forward_fp8 / moe_forward_host_fp8.
     """
 
     def __init__(self, cfg: MoeCfg, weights: dict, max_tokens: int, device="cuda", host_io=False):
@@ -322,19 +325,25 @@ class MoELayer:
         w = self.w
         return (w["W_r"], w.get("b"), w["W1"], w["W3"], w["W2"], w.get("Ws1"), w.get("Ws3"), w.get("Ws2"))
 
+    @property
+    def fp8(self) -> bool:
+        return isinstance(self.w["W1"], (tuple, list))
+
     def __call__(self, x, y=None, topk_idx_out=None, gates_out=None, stream=None):
         import torch
         T = x.shape[0]
         assert T <= self.max_tokens
         if y is None:
             y = torch.empty_like(x)
-        forward(self.cfg, T, x, *self._wargs(), y, self.ws, topk_idx_out, gates_out, stream=stream)
+        fwd = forward_fp8 if self.fp8 else forward
+        fwd(self.cfg, T, x, *self._wargs(), y, self.ws, topk_idx_out, gates_out, stream=stream)
         return y
 
     def forward_host(self, x_host, y_host, stream=None):
         T = x_host.shape[0]
         assert T <= self.max_tokens
-        forward_host(self.cfg, T, x_host, *self._wargs(), y_host, self.ws, stream=stream)
+        fwd = forward_host_fp8 if self.fp8 else forward_host
+        fwd(self.cfg, T, x_host, *self._wargs(), y_host, self.ws, stream=stream)
         return y_host
 
     def device_status(self, T=None, stream=None) -> int:

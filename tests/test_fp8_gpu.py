@@ -177,3 +177,24 @@ def test_fp8_host_entry_matches_device_entry():
     assert torch.equal(y2h, y2_dev.cpu())
     assert moe.device_status(cfg, T2, ws) == 0
     moe.workspace_release(ws)
+
+
+def test_moelayer_runs_fp8_weights():
+    """MoELayer takes (codes, scales) expert weights and runs the FP8 entry
+    points, device and host-buffer, with the same bits as moe_forward_fp8."""
+    s = SMALL["fp8_v3_like"]
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    y_dev, _, _ = run_fp8(s, w, x)
+    layer = moe.MoELayer(cfg_of(s), w, max_tokens=s.T, host_io=True)
+    assert layer.fp8
+    y = layer(x)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_dev)
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    layer.forward_host(xh, yh)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y_dev.cpu())
+    assert layer.device_status() == 0
+    moe.workspace_release(layer.ws)
