@@ -106,16 +106,6 @@ MOE_DEV uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank) {
   return r;
 }
 
-MOE_DEV void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-
-// Arrive (release, cluster scope) on an mbarrier that may live in another CTA.
-MOE_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
 // 4-byte store into shared memory of a CTA of the cluster that completes 4
 // transaction bytes on an mbarrier of that CTA (its complete_tx has release
 // semantics at cluster scope). The issuing thread does not wait for it.

@@ -34,7 +34,8 @@
 // CTA roles (320 threads, one CTA per SM, persistent; the same roles in both
 // CTAs of a pair except the MMA issuer, which only the first CTA has):
 //   warp 0      TMA producer (one lane). In CTA 0 it also takes unit ids and
-//               hands them to both CTAs through shared-memory rings. Stages
+//               hands them to both CTAs through shared-memory rings (the
+//               peer's by an asynchronous store, see below). Stages
 //               are variable-size pieces of a 208 KB byte ring: per 64-wide
 //               K block, 32 KB of weights (two 128-row boxes) and one token
 //               box of 32, 64 or 128 rows (4 / 8 / 16 KB; the TMA engine's
@@ -58,6 +59,11 @@
 // dequantise each stage's codes exactly into bf16 in tensor memory, and the
 // pair MMAs read A from there and B from the ring (kind::f16 as above); four
 // epilogue warps, one per quadrant.
+// Every signal from one CTA of the pair to the other (a unit id, the
+// release of a unit-ring slot or of an accumulator, an FP8 slot report) is
+// an asynchronous store that completes transaction bytes on the receiving
+// CTA's mbarrier (st.async), so no thread waits for a cross-CTA arrive; the
+// MMA commits reach both CTAs' barriers by multicast.
 // Every mbarrier wait is bounded; on a timeout a CTA records
 // MOE_DEV_WAIT_TIMEOUT, drains its own copies and MMAs (bounded again),
 // frees its tensor memory and exits.
