@@ -198,3 +198,15 @@ def test_moelayer_runs_fp8_weights():
     assert torch.equal(yh, y_dev.cpu())
     assert layer.device_status() == 0
     moe.workspace_release(layer.ws)
+
+
+def test_fp8_token_permutation_equivariance_bitwise():
+    """Permuting the tokens permutes the FP8 path's outputs bit for bit."""
+    s = SMALL["fp8_ragged"]
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    y, idx, _ = run_fp8(s, w, x)
+    perm = torch.randperm(s.T, generator=torch.Generator().manual_seed(9))
+    yp, idxp, _ = run_fp8(s, w, x[perm.cuda()].contiguous())
+    assert np.array_equal(idxp, idx[perm.numpy()])
+    assert torch.equal(yp, y[perm.cuda()])

@@ -410,3 +410,22 @@ def test_nonfinite_token_is_flagged_and_isolated():
         if use_forward:
             yk, y0k = t2np64(y)[keep], t2np64(y0)[keep]
             check_outputs(yk, y0k, "bf16", "clean tokens next to a NaN token")
+
+
+@pytest.mark.parametrize("name", ["softmax_ragged", "v3_prefill_bf16"])
+def test_token_permutation_equivariance_bitwise(name):
+    """Each token's output is computed in an order fixed by its own row alone
+    (router K order, the per-element MMA reduction over K, the combine's
+    ascending expert order), so permuting the tokens permutes the outputs,
+    the routing and the gates bit for bit -- although every expert's token
+    rows, MMA tiles and chunks change."""
+    s = SMALL[name] if name in SMALL else mi.SHAPES[name]
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    y, idx, gates = run_forward(s, w, x)
+    perm = torch.randperm(s.T, generator=torch.Generator().manual_seed(7))
+    yp, idxp, gatesp = run_forward(s, w, x[perm.cuda()].contiguous())
+    p = perm.numpy()
+    assert np.array_equal(idxp, idx[p])
+    assert np.array_equal(gatesp, gates[p])
+    assert torch.equal(yp, y[perm.cuda()])
