@@ -77,7 +77,10 @@ enum {
   MOE_DEV_NONFINITE = 1u << 4       /* a token's router logits or keys were NaN or infinite
                                        (non-finite x, W_r or b); it still gets top_k distinct
                                        experts in [0, n_routed), chosen arbitrarily, and the
-                                       other tokens are unaffected */
+                                       other tokens are unaffected */,
+  MOE_DEV_BOUNDS = 1u << 5          /* a bounds check of the debug build (compiled with
+                                       -DMOE_DEBUG_BOUNDS, libmoe_b200_debug.so) failed; the
+                                       checked access was skipped. Never set by the release build */
 };
 
 /*

@@ -9,6 +9,7 @@ missing or the call fails, an exception is raised.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -56,6 +57,20 @@ class MoeError(RuntimeError):
 
 
 _lib = None
+DEBUG_LIB_PATH = os.path.join(_HERE, "libmoe_b200_debug.so")
+
+
+@contextlib.contextmanager
+def using_library(path: str):
+    """Route every call of the binding through the library at `path` (e.g.
+    DEBUG_LIB_PATH, the bounds-checked build) inside the with-block."""
+    global _lib, LIB_PATH
+    saved = (_lib, LIB_PATH)
+    _lib, LIB_PATH = None, path
+    try:
+        yield lib()
+    finally:
+        _lib, LIB_PATH = saved
 
 
 def lib() -> ctypes.CDLL:

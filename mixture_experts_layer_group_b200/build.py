@@ -1,6 +1,9 @@
-"""Build the sm_100a library libmoe_b200.so in-tree with nvcc."""
+"""Build the sm_100a library in-tree with nvcc: libmoe_b200.so, and the
+bounds-checked debug build libmoe_b200_debug.so (-DMOE_DEBUG_BOUNDS: device
+checks before indexed accesses record MOE_DEV_BOUNDS and skip the access)."""
 from __future__ import annotations
 
+import concurrent.futures as cf
 import os
 import subprocess
 import sys
@@ -8,6 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe_b200.so")
+LIB_DEBUG = os.path.join(HERE, "libmoe_b200_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 SOURCES = ["moe_abi.cu", "router.cu", "tensor_map.cu", "dispatch.cu", "combine.cu", "expert_tc.cu", "expert_simt.cu",
            "route_noalloc.cu", "bias_update.cu", "selftest.cu"]
@@ -20,27 +24,32 @@ def _deps():
         os.path.join(HERE, "..", "include", "moe_b200.h")]
 
 
-def up_to_date() -> bool:
-    return os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(d) for d in _deps())
+def up_to_date(debug: bool = False) -> bool:
+    lib = LIB_DEBUG if debug else LIB
+    return os.path.exists(lib) and all(os.path.getmtime(lib) >= os.path.getmtime(d) for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    objdir = os.path.join(HERE, "_build")
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(debug):
+        return lib
+    objdir = os.path.join(HERE, "_build_debug" if debug else "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
-    for src in SOURCES:
+    flags = FLAGS + (["-DMOE_DEBUG_BOUNDS"] if debug else [])
+
+    def compile_one(src):
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
-        cmd = [NVCC, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+        cmd = [NVCC, *flags, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.check_call(cmd)
-        objs.append(obj)
-    subprocess.check_call([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs, "-o", LIB])
-    return LIB
+        return obj
+
+    with cf.ThreadPoolExecutor(max_workers=min(len(SOURCES), os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(compile_one, SOURCES))
+    subprocess.check_call([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs, "-o", lib])
+    return lib
 
 
 if __name__ == "__main__":
-    build(force=True, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force=True, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

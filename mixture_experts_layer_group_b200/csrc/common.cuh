@@ -449,4 +449,15 @@ MOE_DEV void set_status(unsigned* status, unsigned bits) {
   if (status) atomicOr(status, bits);
 }
 
+// Bounds checks of the debug build (-DMOE_DEBUG_BOUNDS): MOE_IN_BOUNDS(cond,
+// status) is cond, and when cond is false it also records MOE_DEV_BOUNDS, so
+// the caller skips the access it guards. The release build compiles it to
+// true: its indices are correct by construction, and the debug build's test
+// checks that no check fires on the same inputs.
+#ifdef MOE_DEBUG_BOUNDS
+#define MOE_IN_BOUNDS(cond, status) ((cond) ? true : (::moe::set_status((status), MOE_DEV_BOUNDS), false))
+#else
+#define MOE_IN_BOUNDS(cond, status) true
+#endif
+
 }  // namespace moe

@@ -83,9 +83,11 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) chunk_kernel(ChunkArgs a) {
         below += (my[s] >= 0 && my[s] < e) ? 1 : 0;
       }
       const int32_t flat = (int32_t)(t * a.k + slot);
-      a.perm[pos] = flat;
-      a.slot_pos[t * a.k + below] = pos;
-      if (a.gates) a.gate_perm[pos] = a.gates[flat];
+      if (MOE_IN_BOUNDS(pos >= 0 && (int64_t)pos < a.T * a.k && below < a.k, a.status)) {
+        a.perm[pos] = flat;
+        a.slot_pos[t * a.k + below] = pos;
+        if (a.gates) a.gate_perm[pos] = a.gates[flat];
+      }
     }
   }
   if (!kScatter) {
@@ -220,13 +222,17 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a, int32_t* chunk_b
 template <typename TV, int KMAX>
 __global__ void __launch_bounds__(256) gather_kernel(const TV* __restrict__ x,
                                                      const int32_t* __restrict__ slot_pos, int64_t T,
-                                                     int k, int vecs, TV* __restrict__ x_perm) {
+                                                     int k, int vecs, TV* __restrict__ x_perm,
+                                                     unsigned* status) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
     int32_t dst[KMAX];
 #pragma unroll
-    for (int s = 0; s < KMAX; ++s) dst[s] = s < k ? __ldg(slot_pos + t * k + s) : -1;
+    for (int s = 0; s < KMAX; ++s) {
+      dst[s] = s < k ? __ldg(slot_pos + t * k + s) : -1;
+      if (dst[s] >= 0 && !MOE_IN_BOUNDS((int64_t)dst[s] < T * k, status)) dst[s] = -1;
+    }
     const TV* src = x + t * vecs;
     for (int v = lane; v < vecs; v += 32) {
       const TV val = __ldg(src + v);
@@ -317,17 +323,18 @@ cudaError_t launch_dispatch(const Problem& p, const DispatchBuffers& db, int bm,
 }
 
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* slot_pos, void* x_perm,
-                          cudaStream_t s) {
+                          unsigned* status, cudaStream_t s) {
   if (p.R == 0) return cudaSuccess;
   const int vecs = (int)((int64_t)p.d * p.elem / 16);
   const int64_t want = (p.T + 7) / 8;
   const int64_t cap = (int64_t)device_sm_count() * 16;
   const unsigned blocks = (unsigned)(want < cap ? want : cap);
   if (p.k <= 8)
-    gather_kernel<uint4, 8><<<blocks, 256, 0, s>>>((const uint4*)x, slot_pos, p.T, p.k, vecs, (uint4*)x_perm);
+    gather_kernel<uint4, 8><<<blocks, 256, 0, s>>>((const uint4*)x, slot_pos, p.T, p.k, vecs, (uint4*)x_perm,
+                                                   status);
   else
     gather_kernel<uint4, kMaxTopK><<<blocks, 256, 0, s>>>((const uint4*)x, slot_pos, p.T, p.k, vecs,
-                                                          (uint4*)x_perm);
+                                                          (uint4*)x_perm, status);
   return cudaGetLastError();
 }
 

@@ -188,6 +188,11 @@ struct TcParams {
   const uint8_t* s1_shared;
   int sblocks_routed, sblocks_shared;
   int chunk_rows;                // token rows of a unit at most (Plan::kChunk)
+  // rows of the token operand, weight and output tensors (routed | shared
+  // group), for the debug build's bounds checks
+  int64_t tok_rows_routed, tok_rows_shared;
+  int64_t a_rows_routed, a_rows_shared;
+  int64_t out_rows_routed, out_rows_shared;
 };
 
 struct Unit {
@@ -522,6 +527,14 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         const uint32_t tx = PL::kABytes + nbox * kBoxBytes;
         const int rowA = (shared ? 0 : un.g * p.a_rows_per_expert) + un.f * p.tile_cols + rank_rows;
         const int rowB = __ldg(p.grp_row0 + un.g) + un.tok0 + (int)rank * half_n;
+        // the unit's rows lie inside the group and its tensors (TMA clips a
+        // box that reaches past them, and the last column tile of a matrix
+        // whose height is not a multiple of the tile may start past it)
+        (void)MOE_IN_BOUNDS(un.ntok >= 1 && un.ntok <= p.chunk_rows && un.tok0 >= 0 &&
+                                __ldg(p.grp_row0 + un.g) + un.tok0 + un.ntok <=
+                                    (shared ? p.tok_rows_shared : p.tok_rows_routed) &&
+                                rowA >= 0 && rowA < (shared ? p.a_rows_shared : p.a_rows_routed) + p.tile_cols,
+                            p.status);
         const CUtensorMap* ta0 = shared ? &p.a0_shared : &p.a0_routed;
         const CUtensorMap* ta1 = MODE == kSwiGLU ? (shared ? &p.a1_shared : &p.a1_routed) : ta0;
         const CUtensorMap* tb = shared ? &p.b_shared[tmap] : &p.b_routed[tmap];
@@ -535,6 +548,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
           }
           off_of[s] = pos;
           head = pos + tx;
+          (void)MOE_IN_BOUNDS(pos + tx <= (uint32_t)kRingBytes, p.status);
           sh.slot_off[s] = pos;
           uint8_t* a_dst = smem + pos;
           uint8_t* b_dst = a_dst + PL::kABytes;
@@ -584,6 +598,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         const uint32_t idesc = idesc_bf16_f32(256, (uint32_t)n);
         uint32_t mask, base, stride;
         plan.place(n, mask, base, stride);
+        (void)MOE_IN_BOUNDS(n <= p.chunk_rows + PL::kTokAlign && base + stride + n <= PL::kAccCols, p.status);
         plan.advance(n);
         for (int b = 0; b < 2 && ok; ++b)
           if ((mask >> b) & 1u) {
@@ -719,7 +734,9 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
           const int64_t row = row_base + tok;
           // gate of this lane's token, spread to the lanes that hold it below
           float my_gate = 1.0f;
-          if (MODE == kGateDown && !shared && p.gate_perm && tok < un.ntok) my_gate = __ldg(p.gate_perm + row);
+          if (MODE == kGateDown && !shared && p.gate_perm && tok < un.ntok &&
+              MOE_IN_BOUNDS(row < p.tok_rows_routed, p.status))
+            my_gate = __ldg(p.gate_perm + row);
           // The block (32 features = this quadrant's TMEM lanes, x 32 tokens =
           // columns j0..j0+31) in the m16n8 layout: lane half hf and column
           // group r give this thread features 16 hf + 8 e + lane / 4 (e = 0, 1)
@@ -780,6 +797,7 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
+              (void)MOE_IN_BOUNDS(row_base + j0 < (shared ? p.out_rows_shared : p.out_rows_routed), p.status);
               tma_store_2d(shared ? &p.o_shared : &p.o_routed, tile, c0,
                            (int)(row_base + j0) + (shared ? p.out_row0_shared : 0));
               bulk_commit_group();
@@ -791,7 +809,11 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
             for (int c = 0; c < 4; ++c)
               rowv[c] = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(tile) + lane * 64 +
                                                         ((c ^ ((lane >> 1) & 3)) << 4));
-            if (tok < un.ntok) store_row32(out_base + row * ld + c0, cols - c0, rowv);
+            // (columns at or past the matrix's width belong to a tile that
+            // reaches past it: nothing to store)
+            if (tok < un.ntok && c0 < cols &&
+                MOE_IN_BOUNDS(row < (shared ? p.out_rows_shared : p.out_rows_routed), p.status))
+              store_row32(out_base + row * ld + c0, cols - c0, rowv);
           }
         }
       }
@@ -881,6 +903,8 @@ __global__ void __launch_bounds__(Plan<FP8>::kThreads, 1) expert_gemm_tc_kernel(
         const int kb = kc >> 1;  // 64-wide K block -> 128-wide scale block
         const int sb = __shfl_sync(0xffffffffu, kb < 32 ? sL : sH, kb & 31);
         const uint32_t raw = smem_u32(smem) + *reinterpret_cast<volatile uint32_t*>(&sh.slot_off[s]);
+        (void)MOE_IN_BOUNDS(*reinterpret_cast<volatile uint32_t*>(&sh.slot_off[s]) + kA8Bytes <= (uint32_t)kRingBytes,
+                            p.status);
         const uint32_t src = raw + row * kBK;
         uint4 wv[4];
 #pragma unroll
@@ -1046,6 +1070,12 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g1.sblocks_routed = (int)((int64_t)p.N * p.F / kFp8Block);
   g1.sblocks_shared = p.nsF / kFp8Block;
   g1.chunk_rows = cm;
+  g1.tok_rows_routed = p.R;
+  g1.tok_rows_shared = p.T;
+  g1.a_rows_routed = (int64_t)p.N * p.F;
+  g1.a_rows_shared = p.nsF;
+  g1.out_rows_routed = p.R;
+  g1.out_rows_shared = p.T;
   const int64_t max_cols1 = p.F > p.nsF ? p.F : p.nsF;
   const int64_t units1 = chunks_bound * ((max_cols1 + kTcBN1 - 1) / kTcBN1);
   const int grid1 = (int)(units1 < sms ? units1 : sms);
@@ -1084,6 +1114,12 @@ cudaError_t launch_expert_gemms_tc(const Problem& p, const GemmArgs& a, cudaStre
   g2.sblocks_routed = (int)((int64_t)p.N * p.d / kFp8Block);
   g2.sblocks_shared = p.d / kFp8Block;
   g2.chunk_rows = cm;
+  g2.tok_rows_routed = p.R;
+  g2.tok_rows_shared = p.T;
+  g2.a_rows_routed = (int64_t)p.N * p.d;
+  g2.a_rows_shared = p.d;
+  g2.out_rows_routed = p.R;
+  g2.out_rows_shared = p.T;
   const int64_t units2 = chunks_bound * ((p.d + kTcBN2 - 1) / kTcBN2);
   const int grid2 = (int)(units2 < sms ? units2 : sms);
   // the down GEMM overlaps the SwiGLU GEMM's drain unless an event must be

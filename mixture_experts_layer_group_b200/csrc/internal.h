@@ -114,8 +114,9 @@ cudaError_t launch_ep_reorder(const int32_t* counts, int W, int E, int64_t row_b
                               bool to_expert_major, cudaStream_t s);
 
 // x_perm[slot_pos[t, s]] = x[t] for every placed (token, slot) pair
+// (status: the workspace's device status word, for the debug build's bounds checks)
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* slot_pos, void* x_perm,
-                          cudaStream_t s);
+                          unsigned* status, cudaStream_t s);
 
 struct GemmArgs {
   const void* x;        // [T, d]

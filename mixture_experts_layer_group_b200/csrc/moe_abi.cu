@@ -191,7 +191,7 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
                                   tc ? kTcBN2 : kSimtBN, s);
   if (e == cudaSuccess) e = mark_stage(2, s);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = launch_gather(p, x, db.slot_pos, at<void>(ws, L.x_perm), s);
+  e = launch_gather(p, x, db.slot_pos, at<void>(ws, L.x_perm), db.status, s);
   if (e == cudaSuccess) e = mark_stage(3, s);
   if (e != cudaSuccess) return cuda_fail(e);
   GemmArgs ga;
@@ -662,7 +662,7 @@ moe_status moe_dispatch_rows(const moe_cfg* cfg, int64_t T, const int32_t* topk_
   cudaError_t e = cudaMemsetAsync(db.status, 0, 4, s);
   if (e == cudaSuccess)
     e = launch_dispatch(p, db, tc ? kTcBM : kSimtBM, tc ? kTcBN1 : kSimtBN, tc ? kTcBN2 : kSimtBN, s);
-  if (e == cudaSuccess) e = launch_gather(p, x, slot_pos, x_perm, s);
+  if (e == cudaSuccess) e = launch_gather(p, x, slot_pos, x_perm, db.status, s);
   if (e == cudaSuccess) e = note_device_use(ws, s);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }

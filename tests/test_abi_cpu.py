@@ -50,6 +50,19 @@ def test_binding_declares_argument_types(L):
         assert getattr(L, name).argtypes is not None, name
 
 
+def test_debug_build_exports_the_same_abi():
+    """The bounds-checked debug build (-DMOE_DEBUG_BOUNDS) compiles, loads and
+    exports exactly the header's functions, like the release build."""
+    path = moe_build.build(debug=True)
+    assert path == moe.DEBUG_LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    assert {s for s in syms if s.startswith("moe_")} == set(header_functions())
+    with moe.using_library(path) as D:
+        assert D.moe_status_string(0).decode() == moe.lib().moe_status_string(0).decode()
+    assert moe.LIB_PATH != path
+
+
 def test_cfg_struct_matches_header():
     src = open(HEADER).read()
     body = re.search(r"typedef struct moe_cfg \{(.*?)\} moe_cfg;", src, flags=re.S).group(1)
