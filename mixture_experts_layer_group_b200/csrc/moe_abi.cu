@@ -6,10 +6,35 @@
 #include <mutex>
 #include <unordered_map>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
+
+// NVTX ranges for timeline tools: one for a layer forward and, nested in it,
+// one per stage (the host-side enqueue of that stage's launches, which a
+// timeline tool ties to the kernels). With no tool attached an NVTX call
+// costs a check of a function pointer.
+class NvtxStages {
+ public:
+  explicit NvtxStages(const char* call) { nvtxRangePushA(call); }
+  void stage(const char* name) {
+    if (open_) nvtxRangePop();
+    nvtxRangePushA(name);
+    open_ = true;
+  }
+  ~NvtxStages() {
+    if (open_) nvtxRangePop();
+    nvtxRangePop();
+  }
+  NvtxStages(const NvtxStages&) = delete;
+  NvtxStages& operator=(const NvtxStages&) = delete;
+
+ private:
+  bool open_ = false;
+};
 
 namespace {
 thread_local int32_t g_last_cuda_error = 0;
@@ -176,21 +201,25 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
                           const void* Ws1, const void* Ws3, const void* Ws2, void* y,
                           int32_t* idx_out, float* gates_out, void* ws, cudaStream_t s,
                           const Fp8Scales* fp8 = nullptr) {
+  NvtxStages nv(fp8 ? "moe_forward_fp8" : "moe_forward");
   int32_t* idx = at<int32_t>(ws, L.idx);
   float* gates = at<float>(ws, L.gates);
   cudaError_t e0 = cudaMemsetAsync(at<void>(ws, L.status), 0, 4, s);
   if (e0 == cudaSuccess) e0 = mark_stage(0, s);
   if (e0 != cudaSuccess) return cuda_fail(e0);
+  nv.stage("moe.router");
   moe_status st = run_router(p, L, x, W_r, b, idx, gates, ws, s);
   if (st != MOE_OK) return st;
   if ((e0 = mark_stage(1, s)) != cudaSuccess) return cuda_fail(e0);
   const bool tc = p.dtype == MOE_BF16;
   DispatchBuffers db = dispatch_buffers(L, ws, idx, gates);
+  nv.stage("moe.dispatch");
   // unit tables for the GEMMs: FP8 weights cut groups into chunks of at most kTcBM8 rows
   cudaError_t e = launch_dispatch(p, db, tc ? (fp8 ? kTcBM8 : kTcBM) : kSimtBM, tc ? kTcBN1 : kSimtBN,
                                   tc ? kTcBN2 : kSimtBN, s);
   if (e == cudaSuccess) e = mark_stage(2, s);
   if (e != cudaSuccess) return cuda_fail(e);
+  nv.stage("moe.gather");
   e = launch_gather(p, x, db.slot_pos, at<void>(ws, L.x_perm), db.status, s);
   if (e == cudaSuccess) e = mark_stage(3, s);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -222,10 +251,12 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
     ga.Ws3s = p.ns ? fp8->s[4] : nullptr;
     ga.Ws2s = p.ns ? fp8->s[5] : nullptr;
   }
+  nv.stage("moe.expert_gemms");
   e = tc ? launch_expert_gemms_tc(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr)
          : launch_expert_gemms_simt(p, ga, s, g_stage_events_on ? g_stage_events[4] : nullptr);
   if (e == cudaSuccess) e = mark_stage(5, s);
   if (e != cudaSuccess) return cuda_fail(e);
+  nv.stage("moe.combine");
   e = launch_combine(p, ga.y_rows, db.slot_pos, y, s);
   if (e == cudaSuccess) e = mark_stage(6, s);
   if (e != cudaSuccess) return cuda_fail(e);
