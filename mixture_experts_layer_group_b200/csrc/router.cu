@@ -252,18 +252,32 @@ __global__ void __launch_bounds__(256) router_select_kernel(SelectArgs a) {
   const int N = a.N;
   const float* zrow = a.logits + t * N;
 
+  // z = plane 0 + plane 1 + ... in this order for every expert; the loads
+  // of four planes are issued before their adds, so a token's 4 V loads are
+  // in flight together instead of one dependent L2 round trip per plane
+  const int64_t plane = a.T * N;
   float s[V], key[V];
 #pragma unroll
-  for (int j = 0; j < V; ++j) {
-    int e = 32 * j + lane;
-    if (e < N) {
-      float z = zrow[e];
-      for (int sp = 1; sp < a.S; ++sp) z += zrow[(int64_t)sp * a.T * N + e];  // fixed order
-      s[j] = z;
-    } else {
-      s[j] = -INFINITY;
-    }
+  for (int j = 0; j < V; ++j) s[j] = 32 * j + lane < N ? zrow[32 * j + lane] : 0.f;
+  int sp = 1;
+  for (; sp + 4 <= a.S; sp += 4) {
+    float v[4][V];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int j = 0; j < V; ++j) v[q][j] = 32 * j + lane < N ? zrow[(sp + q) * plane + 32 * j + lane] : 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int j = 0; j < V; ++j) s[j] += v[q][j];
   }
+  for (; sp < a.S; ++sp) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) s[j] += 32 * j + lane < N ? zrow[sp * plane + 32 * j + lane] : 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < V; ++j)
+    if (32 * j + lane >= N) s[j] = -INFINITY;
   if (a.score_fn == MOE_SOFTMAX) {
     float m = -INFINITY;
 #pragma unroll
