@@ -216,17 +216,22 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a, int32_t* chunk_b
   }
 }
 
-// x_perm[slot_pos[t, s]] = x[t] for every placed pair: one warp per token
-// reads its row once and writes it to each of its k permuted rows, so x is
-// read from HBM once (a pair left at -1 by an invalid index is skipped).
+// x_perm[slot_pos[t, s]] = x[t] for every placed pair: a warp reads its
+// part of a token's row once and writes it to each of the token's k permuted
+// rows, so x is read from HBM once (a pair left at -1 by an invalid index is
+// skipped). A row is split into `parts` column ranges handled by separate
+// warps when there are few tokens (decode), so the copy spreads over the GPU.
 template <typename TV, int KMAX>
 __global__ void __launch_bounds__(256) gather_kernel(const TV* __restrict__ x,
                                                      const int32_t* __restrict__ slot_pos, int64_t T,
-                                                     int k, int vecs, TV* __restrict__ x_perm,
+                                                     int k, int vecs, int parts, TV* __restrict__ x_perm,
                                                      unsigned* status) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < T * parts; w += warps) {
+    const int64_t t = w / parts;
+    const int part = (int)(w % parts);
+    const int v0 = (int)((int64_t)part * vecs / parts), v1 = (int)((int64_t)(part + 1) * vecs / parts);
     int32_t dst[KMAX];
 #pragma unroll
     for (int s = 0; s < KMAX; ++s) {
@@ -234,7 +239,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const TV* __restrict__ x,
       if (dst[s] >= 0 && !MOE_IN_BOUNDS((int64_t)dst[s] < T * k, status)) dst[s] = -1;
     }
     const TV* src = x + t * vecs;
-    for (int v = lane; v < vecs; v += 32) {
+    for (int v = v0 + lane; v < v1; v += 32) {
       const TV val = __ldg(src + v);
 #pragma unroll
       for (int s = 0; s < KMAX; ++s)
@@ -326,14 +331,21 @@ cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* slot_p
                           unsigned* status, cudaStream_t s) {
   if (p.R == 0) return cudaSuccess;
   const int vecs = (int)((int64_t)p.d * p.elem / 16);
-  const int64_t want = (p.T + 7) / 8;
-  const int64_t cap = (int64_t)device_sm_count() * 16;
+  const int sms = device_sm_count();
+  // warps per token: enough for about 8 warps per SM, at most 8 and at least
+  // 32 vectors (one per lane) per part
+  int64_t parts = ((int64_t)sms * 8 + p.T - 1) / p.T;
+  if (parts > 8) parts = 8;
+  if (parts > vecs / 32) parts = vecs / 32;
+  if (parts < 1) parts = 1;
+  const int64_t want = (p.T * parts + 7) / 8;
+  const int64_t cap = (int64_t)sms * 16;
   const unsigned blocks = (unsigned)(want < cap ? want : cap);
   if (p.k <= 8)
-    gather_kernel<uint4, 8><<<blocks, 256, 0, s>>>((const uint4*)x, slot_pos, p.T, p.k, vecs, (uint4*)x_perm,
-                                                   status);
+    gather_kernel<uint4, 8><<<blocks, 256, 0, s>>>((const uint4*)x, slot_pos, p.T, p.k, vecs, (int)parts,
+                                                   (uint4*)x_perm, status);
   else
-    gather_kernel<uint4, kMaxTopK><<<blocks, 256, 0, s>>>((const uint4*)x, slot_pos, p.T, p.k, vecs,
+    gather_kernel<uint4, kMaxTopK><<<blocks, 256, 0, s>>>((const uint4*)x, slot_pos, p.T, p.k, vecs, (int)parts,
                                                           (uint4*)x_perm, status);
   return cudaGetLastError();
 }
