@@ -29,12 +29,27 @@ Readings where the pages are silent (each is listed in the design notes):
   * the residual is not part of Delta_ffn.
 No value is rounded: inputs are widened exactly to fp64 and stay there.
 
-Pins (tests/test_oracle_pins.py): selection by brute force over all subsets,
-the printed parameter and combination counts, closed forms, and identities
-(segmentation, shared fusion, dense ceiling, identical experts, GShard
-special case). The pages print no worked layer output, so output values are
-pinned only through those identities and closed forms: beyond them, parity
-unpinned.
+Pins (tests/test_oracle_pins.py), by function:
+  * softmax / sigmoid / silu: closed forms and value pins (sigma(ln 3) = 3/4,
+    silu(ln 3) = 3/4 ln 3).
+  * router_logits: the product with each router row written out.
+  * route: top-k against brute force over all subsets, with and without the
+    group limit; tie flags; normalised gates summing to route_scale; the bias
+    steering the selection but not the gates.
+  * gates_for: a hand-computed example; equal to route's gates.
+  * permutation: the sorted (expert, token) pairs.
+  * bias_update: a hand example and its sign / magnitude properties.
+  * expert_ffn / forward / gate_matrix: the SwiGLU bilinear identity, the
+    segmentation and shared-fusion identities, the dense ceiling, identical
+    experts (route_scale x FFN + shared), the GShard two-expert closed form,
+    expert and token permutation equivariance, the idx_override path on the
+    routing's own selection and on a hand-built exact tie.
+  * e4m3_value / dequant_fp8: every code against the OCP E4M3 definition; a
+    hand-computed 128 x 128 block example.
+  * expert_params / router_params / block_params / routing_combinations /
+    flops_per_token: the pages' printed counts.
+The pages print no worked layer output, so output values are pinned only
+through those identities and closed forms: beyond them, parity unpinned.
 """
 from __future__ import annotations
 
