@@ -2,7 +2,7 @@
 // and the row gather that feeds the grouped GEMMs. This replaces the quoted
 // MoE.forward's bincount(...).tolist() and per-expert torch.where loop
 // ("DeepSeek-V3.2-Exp · Mixture of experts", quoted forward excerpt) with
-// three small kernels and no host round trip.
+// three small kernels (one for decode-sized batches) and no host round trip.
 //
 // Bit-exact by construction: a warp owns 32 consecutive tokens; for each
 // expert it forms a ballot of the tokens that chose it, so a pair's rank
@@ -35,10 +35,9 @@ struct ChunkArgs {
 // within the chunk is the popcount of the lower lanes. Pass 0 writes the
 // per-chunk counts, pass 1 places every pair.
 template <bool kScatter>
-__global__ void __launch_bounds__(32 * kWarpsPerCta) chunk_kernel(ChunkArgs a) {
+MOE_DEV void chunk_pass(const ChunkArgs& a, int64_t gw) {
   const int lane = threadIdx.x & 31;
   const int W = (a.N + 31) / 32;
-  const int64_t gw = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   const int64_t n_chunks = (a.T + 31) / 32;
   if (gw >= n_chunks * W) return;
   const int64_t c = gw / W;
@@ -96,6 +95,11 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) chunk_kernel(ChunkArgs a) {
   }
 }
 
+template <bool kScatter>
+__global__ void __launch_bounds__(32 * kWarpsPerCta) chunk_kernel(ChunkArgs a) {
+  chunk_pass<kScatter>(a, (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5));
+}
+
 // Exclusive scan of v over the whole block (blockDim.x a multiple of 32,
 // at most 1024); returns the prefix and writes the block total to *total.
 MOE_DEV int block_exclusive_scan(int v, int* total) {
@@ -142,9 +146,9 @@ struct ScanArgs {
   int32_t* unit_base2;
 };
 
-// One CTA of 1024 threads: per-expert totals and chunk bases, offsets, and the
-// GEMM unit tables (groups 0..N-1 routed, group N the shared MLP).
-__global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a, int32_t* chunk_base) {
+// Run by one CTA of 1024 threads: per-expert totals and chunk bases, offsets,
+// and the GEMM unit tables (groups 0..N-1 routed, group N the shared MLP).
+MOE_DEV void scan_pass(const ScanArgs& a, int32_t* chunk_base) {
   const int tid = threadIdx.x;
   int cnt = 0;
   if (tid < a.N) {
@@ -214,6 +218,30 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a, int32_t* chunk_b
     a.unit_base1[a.N + 1] = tot1;
     a.unit_base2[a.N + 1] = tot2;
   }
+}
+
+__global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a, int32_t* chunk_base) { scan_pass(a, chunk_base); }
+
+// The whole dispatch in one CTA of 1024 threads when every chunk warp fits
+// in it (decode-sized batches): slot_pos reset, the counting pass into shared
+// memory, the scan, and the placing pass -- the same passes as the three
+// kernels above, so the same positions, with one launch instead of three and
+// a memset.
+__global__ void __launch_bounds__(1024) dispatch_small_kernel(ChunkArgs ca, ScanArgs sa) {
+  extern __shared__ int32_t dsm[];  // [n_chunks, N] counts, then [n_chunks, N] bases
+  const int64_t n = ((ca.T + 31) / 32) * ca.N;
+  for (int64_t i = threadIdx.x; i < ca.T * ca.k; i += blockDim.x) ca.slot_pos[i] = -1;
+  ChunkArgs a = ca;
+  a.chunk_counts = dsm;
+  a.chunk_base = dsm + n;
+  const int64_t gw = threadIdx.x >> 5;
+  chunk_pass<false>(a, gw);
+  __syncthreads();
+  ScanArgs s = sa;
+  s.chunk_counts = dsm;
+  scan_pass(s, dsm + n);
+  __syncthreads();
+  chunk_pass<true>(a, gw);
 }
 
 // x_perm[slot_pos[t, s]] = x[t] for every placed pair: a warp reads its
@@ -313,6 +341,13 @@ cudaError_t launch_dispatch(const Problem& p, const DispatchBuffers& db, int bm,
   const unsigned blocks = (unsigned)((warps + kWarpsPerCta - 1) / kWarpsPerCta);
   ChunkArgs ca{db.idx, p.T, p.N, p.k, db.chunk_counts, db.chunk_base, db.gates, db.perm,
                db.slot_pos, db.gate_perm, db.status};
+  const size_t small_smem = (size_t)2 * n_chunks * p.N * sizeof(int32_t);
+  if (warps <= 32 && small_smem <= 48 * 1024) {
+    ScanArgs sa{nullptr, n_chunks, p.T, p.N, p.ns, p.F, p.nsF, p.d, bm, bn1, bn2,
+                db.counts, db.offsets, db.grp_row0, db.grp_rows, db.unit_base1, db.unit_base2};
+    dispatch_small_kernel<<<1, 1024, small_smem, s>>>(ca, sa);
+    return cudaGetLastError();
+  }
   cudaError_t err = cudaMemsetAsync(db.slot_pos, 0xFF, (size_t)p.R * sizeof(int32_t), s);
   if (err != cudaSuccess) return err;
   chunk_kernel<false><<<blocks, 32 * kWarpsPerCta, 0, s>>>(ca);
