@@ -41,6 +41,9 @@ CASES = {
     # a skewed layer: experts with several chunks of the largest unit
     "skewed_chunks": LS("skewed_chunks", T=1024, d=256, n_routed=16, n_shared=1, d_ff=256, top_k=2,
                         score="softmax", seed=41, zipf_s=1.5),
+    # the same on the FP8 path (chunks of its smaller unit)
+    "fp8_skewed_chunks": LS("fp8_skewed_chunks", T=1024, d=256, n_routed=16, n_shared=1, d_ff=256, top_k=2,
+                            score="softmax", seed=42, zipf_s=1.5, wdtype="fp8"),
 }
 
 

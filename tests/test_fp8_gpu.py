@@ -117,6 +117,38 @@ def test_fp8_small_layer_against_oracle(name):
     check_outputs(t2np64(y), ref, "bf16", name)
 
 
+def test_fp8_skewed_routing_many_chunks():
+    """Every token drawn to the same four experts by a large selection bias:
+    each gets T = 1000 rows, seven chunks of equal size on the FP8 path.
+    Bit for bit equal to moe_forward on the dequantised weights (whose
+    chunks are larger) and within tolerance of the oracle."""
+    s = LS("fp8_skewed", T=1000, d=256, n_routed=32, n_shared=1, d_ff=256, top_k=4, score="sigmoid",
+           n_groups=4, topk_groups=2, normalize=True, route_scale=2.5, seed=34, bias=True, wdtype="fp8")
+    hot = [3, 5, 17, 22]
+    bias = np.zeros(s.n_routed, np.float32)
+    bias[hot] = 4.0
+    w = mdev.device_all(s)
+    w["b"] = torch.from_numpy(bias).cuda()
+    x = mdev.device_tensor(s, "x")
+    y, gidx, ggates = run_fp8(s, w, x)
+    assert (np.sort(gidx, axis=1) == hot).all()
+    wb = dict(w)
+    for nm in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2"):
+        q, sc = w[nm]
+        wb[nm] = bf16_device(oracle.dequant_fp8(q.cpu().numpy(), sc.cpu().numpy()))
+    cfg = cfg_of(s)
+    yb = torch.empty_like(x)
+    moe.forward(cfg, s.T, x, wb["W_r"], wb["b"], wb["W1"], wb["W3"], wb["W2"], wb["Ws1"], wb["Ws3"], wb["Ws2"], yb,
+                workspace(cfg, s.T))
+    torch.cuda.synchronize()
+    assert torch.equal(yb, y)
+    h = mi.host_all(s.with_(wdtype="bf16"))
+    ref, r = oracle_forward(s, f64(h["x"]), f64(h["W_r"]), bias.astype(np.float64), expert_fn_fp8(s), shared_fp8(s),
+                            gidx)
+    check_routing(gidx, ggates, r, router_cfg_of(s))
+    check_outputs(t2np64(y), ref, "bf16", s.name)
+
+
 @pytest.mark.parametrize("name", ["v3_decode_fp8", "v3_prefill_fp8"])
 def test_fp8_full_size_every_token(name):
     s = mi.SHAPES[name]

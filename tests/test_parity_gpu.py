@@ -77,6 +77,35 @@ def test_small_layer_full_parity(name):
     full_oracle_check(SMALL[name])
 
 
+@pytest.mark.parametrize("dtype,strength", [("bf16", 4.0), ("bf16", 0.3), ("f32", 4.0)])
+def test_skewed_routing_many_chunks(dtype, strength):
+    """A selection bias that draws (nearly) every token to the same four
+    experts: each of them gets up to T = 1000 rows, so its units split into
+    several chunks of equal size with a ragged last one (the bias moves the
+    selection only, the gates still come from the unbiased scores)."""
+    s = LS("skewed_" + dtype, T=1000, d=256, n_routed=32, n_shared=1, d_ff=192, top_k=4, score="sigmoid",
+           n_groups=4, topk_groups=2, normalize=True, route_scale=2.5, dtype=dtype, seed=21, bias=True)
+    hot = [3, 5, 17, 22]  # two experts in each of groups 0 and 2
+    bias = np.zeros(s.n_routed, np.float32)
+    bias[hot] = strength
+    w = mdev.device_all(s)
+    w["b"] = torch.from_numpy(bias).cuda()
+    x = mdev.device_tensor(s, "x")
+    y, gidx, ggates = run_forward(s, w, x)
+    h = mi.host_all(s)
+    expert = lambda e: (f64(h["W1"][e]), f64(h["W3"][e]), f64(h["W2"][e]))  # noqa: E731
+    shared = (f64(h["Ws1"]), f64(h["Ws3"]), f64(h["Ws2"]))
+    x64, W_r64 = f64(h["x"]), f64(h["W_r"])
+    ref, r = oracle_forward(s, x64, W_r64, bias.astype(np.float64), expert, shared, gidx)
+    check_routing(gidx, ggates, r, router_cfg_of(s))
+    counts = np.bincount(gidx.ravel(), minlength=s.n_routed)
+    if strength >= 1.0:
+        assert (np.sort(gidx, axis=1) == hot).all()
+    else:
+        assert counts[hot].min() > 256 and counts[hot].max() < s.T, counts[hot]
+    check_outputs(t2np64(y), ref, s.dtype, s.name)
+
+
 def test_dispatch_bit_exact_and_edge_cases():
     s = SMALL["v3_like_small"]
     cfg = cfg_of(s)
