@@ -87,6 +87,14 @@ def ncu_traffic(config: str):
     return rec.get("bytes_per_launch")
 
 
+def wait_event(ev, poll_s=0.0005):
+    """Waits for a CUDA event by polling it with short sleeps, which release
+    the interpreter lock, so the clock sampler's thread keeps running while
+    the device works through the timed region."""
+    while not ev.query():
+        time.sleep(poll_s)
+
+
 class ClockSampler:
     """SM clock and clock-event reasons of one GPU, polled through NVML every
     few milliseconds while the timed region runs (nvidia-smi's 200 ms period
@@ -243,6 +251,7 @@ class Layer:
         for _ in range(steps):
             self.step()
         t1.record(self.stream)
+        wait_event(t1)
         torch.cuda.synchronize()
         return t0.elapsed_time(t1) / steps
 
@@ -264,24 +273,33 @@ class Layer:
         return {name: float(np.mean([ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)]))
                 for i, name in enumerate(self.moe.STAGES)}
 
-    def e2e(self, steps, warmup):
-        """ms per step through moe_forward_host: x copied in from pinned host
-        memory and y copied back to it on every step."""
+    def e2e(self, steps, warmup, async_out=True):
+        """ms per step through the host-buffer calls: x copied in from pinned
+        host memory and y copied back to it on every step. async_out: the
+        moe_forward_host(_fp8)_async calls (each step's output copy overlaps
+        the next step; the wait for the last one is inside the timed region),
+        else moe_forward_host(_fp8) (output copy on the caller's stream)."""
         import torch
         xh = self.x.cpu().pin_memory()
-        yh = torch.empty_like(xh).pin_memory()
-        fwd = self.moe.forward_host_fp8 if self.s.wdtype == "fp8" else self.moe.forward_host
-        for _ in range(warmup):
-            fwd(self.cfg, self.s.T, xh, *self.wargs, yh, self.ws, stream=self.stream)
+        yh = [torch.empty_like(xh).pin_memory() for _ in range(2)]
+        fp8 = self.s.wdtype == "fp8"
+        if async_out:
+            fwd = self.moe.forward_host_fp8_async if fp8 else self.moe.forward_host_async
+        else:
+            fwd = self.moe.forward_host_fp8 if fp8 else self.moe.forward_host
+        for i in range(warmup):
+            fwd(self.cfg, self.s.T, xh, *self.wargs, yh[i & 1], self.ws, stream=self.stream)
+        self.moe.host_wait(self.ws, self.stream)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(self.stream)
-        for _ in range(steps):
-            fwd(self.cfg, self.s.T, xh, *self.wargs, yh, self.ws, stream=self.stream)
+        for i in range(steps):
+            fwd(self.cfg, self.s.T, xh, *self.wargs, yh[i & 1], self.ws, stream=self.stream)
+        self.moe.host_wait(self.ws, self.stream)
         e1.record(self.stream)
         torch.cuda.synchronize()
         self.moe.workspace_release(self.ws)
-        return e0.elapsed_time(e1) / steps, xh.numel() * xh.element_size(), yh.numel() * yh.element_size()
+        return e0.elapsed_time(e1) / steps, xh.numel() * xh.element_size(), yh[0].numel() * yh[0].element_size()
 
     def free(self):
         import torch
@@ -325,6 +343,7 @@ def run_ours(args, rank, world, local_rank):
     stage_ms = L.stage_pass(min(args.steps, 20))
     # --- end to end through the host-buffer entry point
     e2e_ms, h2d, d2h = L.e2e(args.steps, max(1, args.warmup // 2))
+    e2e_sync_ms = L.e2e(args.steps, max(1, args.warmup // 2), async_out=False)[0]
     L.free()
 
     # --- the V3 decode layer, timed the same way
@@ -359,9 +378,9 @@ def run_ours(args, rank, world, local_rank):
         Fl.free()
         f8 = (fs, fms, fcounts, fstatus, fstage, fclk.summary())
 
-    vals = [ms, e2e_ms] + ([dec[1]] if dec else []) + ([f8[1]] if f8 else [])
+    vals = [ms, e2e_ms, e2e_sync_ms] + ([dec[1]] if dec else []) + ([f8[1]] if f8 else [])
     vals = max_over_ranks(vals, device="cuda")
-    ms, e2e_ms = vals[0], vals[1]
+    ms, e2e_ms, e2e_sync_ms = vals[0], vals[1], vals[2]
     if rank != 0:
         return None
 
@@ -396,8 +415,12 @@ def run_ours(args, rank, world, local_rank):
                          "GB of expert weights"},
         "e2e": {"value": round(world * s.T / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
-                "api": ("moe_forward_host_fp8" if s.wdtype == "fp8" else "moe_forward_host")
-                       + " (pinned host x in, y out, every step)"},
+                "api": ("moe_forward_host_fp8_async" if s.wdtype == "fp8" else "moe_forward_host_async")
+                       + " (pinned host x in, y out, every step; each step's output copy overlaps the next "
+                         "step, moe_host_wait for the last one inside the timed region)",
+                "sync_ms_per_step": round(e2e_sync_ms, 4),
+                "sync_api": ("moe_forward_host_fp8" if s.wdtype == "fp8" else "moe_forward_host")
+                            + " (output copy on the caller's stream after each step)"},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "roofline": {"bound": "hbm", "kernel": "expert_gemm_tc_kernel<SwiGLU>",
                      "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -420,7 +443,7 @@ def run_ours(args, rank, world, local_rank):
     }
     if dec:
         ds, dms, dcounts, dstatus, dstage, dclocks = dec
-        dms = vals[2]
+        dms = vals[3]
         DA = algorithmic(ds, dcounts)
         dt = dms / 1e3
         d_t_hbm = DA["layer_bytes"] / (peaks["hbm_gbs"] * 1e9)

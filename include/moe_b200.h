@@ -218,16 +218,17 @@ MOE_API moe_status moe_forward_fp8(const moe_cfg* cfg, int64_t T, const void* x,
  * caller synchronises the stream before reading y_host. Weights stay in
  * device memory. Needs moe_workspace_size_host() bytes of workspace.
  * The host-to-device copy runs on a copy stream the library keeps for the
- * workspace (with four events, no device memory; created on the first host
- * call on that workspace, freed by moe_workspace_release or at process exit).
- * x is staged in two slots used by alternate calls, so back-to-back calls
+ * workspace (with a second stream for moe_forward_host_async's output copies
+ * and eight events, no device memory; created on the first host call on that
+ * workspace, freed by moe_workspace_release or at process exit). x and y are
+ * each staged in two slots used by alternate calls, so back-to-back calls
  * with the same T and cfg overlap one call's input copy with the whole of
  * the previous call. A call with another T or cfg, or one that follows a
- * moe_route / moe_dispatch / moe_forward call on the same workspace, waits
- * for the previous call to finish before copying (its staging area may then
- * overlap buffers that call still uses). The output copy stays on `stream`.
- * All calls on one workspace must be ordered: issue them on one stream, or
- * order the streams yourself.
+ * device-buffer call (moe_route, moe_dispatch, moe_forward, ...) on the same
+ * workspace, waits for the previous call to finish before copying (its
+ * staging area may then overlap buffers that call still uses). The output
+ * copy stays on `stream`. All calls on one workspace must be ordered: issue
+ * them on one stream, or order the streams yourself.
  */
 MOE_API moe_status moe_workspace_size_host(const moe_cfg* cfg, int64_t T, size_t* bytes);
 MOE_API moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
@@ -236,10 +237,42 @@ MOE_API moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x
                             void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Frees the copy stream and events that moe_forward_host keeps for the
+ * moe_forward_host with the output copy off `stream`: the forward is
+ * enqueued on `stream` as in moe_forward_host, and y is copied from its
+ * staging slot to y_host on the workspace's output stream once the forward
+ * has written it. A run of calls then overlaps each call's input copy with
+ * the previous call and its output copy with the next call, so it proceeds
+ * at the rate of the forward alone. y_host is complete only after a later
+ * moe_host_wait(ws, s) has been reached by a stream s (synchronise s, or
+ * wait on an event recorded after it, before reading y_host); until then the
+ * caller must neither read nor free it. x_host may be reused once `stream`
+ * has passed the call, as with moe_forward_host. A slot's y is overwritten
+ * two calls later only after its copy out has finished, and every
+ * device-buffer entry point on the workspace (and a host call with another
+ * T or cfg) first waits for the output copies still pending, so calls of
+ * both kinds can be mixed on one workspace. Same arguments, workspace size
+ * and errors as moe_forward_host.
+ */
+MOE_API moe_status moe_forward_host_async(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
+                                          const float* b, const void* W1, const void* W3, const void* W2,
+                                          const void* Ws1, const void* Ws3, const void* Ws2, void* y_host,
+                                          void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Makes `stream` wait (on the device, without blocking the host) until every
+ * output copy that moe_forward_host_async / moe_forward_host_fp8_async have
+ * issued on the workspace at `ws` so far has finished. Returns at once (and
+ * MOE_OK) when the workspace has no asynchronous output copies.
+ * Errors: MOE_ERR_CUDA from the stream wait.
+ */
+MOE_API moe_status moe_host_wait(const void* ws, void* stream);
+
+/*
+ * Frees the copy streams and events that the host-buffer calls keep for the
  * workspace at `ws` (nothing happens if it has none). Call it before freeing
- * or reusing that memory for another purpose; work still queued on the
- * stream completes first. The workspace memory itself belongs to the caller.
+ * or reusing that memory for another purpose; it blocks until the copies
+ * still queued on those streams (which read or write the caller's host
+ * buffers) have finished. The workspace memory itself belongs to the caller.
  * Errors: MOE_ERR_CUDA if the workspace's device cannot be made current.
  */
 MOE_API moe_status moe_workspace_release(const void* ws);
@@ -250,13 +283,21 @@ MOE_API moe_status moe_workspace_release(const void* ws);
  * forward of moe_forward_fp8 (same weights arguments, requirements and
  * results). The workspace is sized by moe_workspace_size_host; the per-
  * workspace state is shared with moe_forward_host and freed by
- * moe_workspace_release.
+ * moe_workspace_release. moe_forward_host_fp8_async is the same with the
+ * output copy of moe_forward_host_async (y_host complete after a later
+ * moe_host_wait).
  */
 MOE_API moe_status moe_forward_host_fp8(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
                                 const float* b, const moe_fp8_matrix* W1, const moe_fp8_matrix* W3,
                                 const moe_fp8_matrix* W2, const moe_fp8_matrix* Ws1,
                                 const moe_fp8_matrix* Ws3, const moe_fp8_matrix* Ws2, void* y_host,
                                 void* ws, size_t ws_bytes, void* stream);
+MOE_API moe_status moe_forward_host_fp8_async(const moe_cfg* cfg, int64_t T, const void* x_host,
+                                              const void* W_r, const float* b, const moe_fp8_matrix* W1,
+                                              const moe_fp8_matrix* W3, const moe_fp8_matrix* W2,
+                                              const moe_fp8_matrix* Ws1, const moe_fp8_matrix* Ws3,
+                                              const moe_fp8_matrix* Ws2, void* y_host, void* ws,
+                                              size_t ws_bytes, void* stream);
 
 /*
  * Reads (and optionally clears) the device-status word of a workspace used

@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ["moe_workspace_size", "moe_workspace_size_host", "moe_route", "moe_dispatch", "moe_forward",
            "moe_forward_fp8", "moe_dispatch_rows", "moe_experts_workspace_size", "moe_experts", "moe_combine",
            "moe_ep_reorder",
-           "moe_forward_host", "moe_forward_host_fp8", "moe_workspace_release", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update", "moe_selftest_wait_timeout",
+           "moe_forward_host", "moe_forward_host_fp8", "moe_forward_host_async", "moe_forward_host_fp8_async",
+           "moe_host_wait", "moe_workspace_release", "moe_device_status", "moe_set_stage_events", "moe_route_noalloc", "moe_bias_update", "moe_selftest_wait_timeout",
            "moe_status_string", "moe_last_cuda_error"]
 STAGES = ["router", "dispatch", "gather", "gemm_swiglu", "gemm_gate", "combine"]
 
@@ -97,6 +98,9 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_fp8.argtypes = [CFG, I64, P, P, P, FP8P, FP8P, FP8P, FP8P, FP8P, FP8P, P, P, P, P, SZ, P]
         L.moe_forward_host.argtypes = [CFG, I64, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.moe_forward_host_fp8.argtypes = [CFG, I64, P, P, P, FP8P, FP8P, FP8P, FP8P, FP8P, FP8P, P, P, SZ, P]
+        L.moe_forward_host_async.argtypes = L.moe_forward_host.argtypes
+        L.moe_forward_host_fp8_async.argtypes = L.moe_forward_host_fp8.argtypes
+        L.moe_host_wait.argtypes = [P, P]
         L.moe_workspace_release.argtypes = [P]
         L.moe_device_status.argtypes = [CFG, I64, P, SZ, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32), P]
         L.moe_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
@@ -287,8 +291,35 @@ def forward_host_fp8(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, 
                                                               ws_bytes, _stream(stream)))
 
 
+def forward_host_async(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, ws_bytes=None,
+                       stream=None):
+    """moe_forward_host with the output copy on the workspace's own stream:
+    y_host is complete after a later host_wait(ws, stream) has been reached."""
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    _check("moe_forward_host_async",
+           lib().moe_forward_host_async(ctypes.byref(cfg), T, _ptr(x_host), _ptr(W_r), _ptr(b), _ptr(W1), _ptr(W3),
+                                        _ptr(W2), _ptr(Ws1), _ptr(Ws3), _ptr(Ws2), _ptr(y_host), _ptr(ws), ws_bytes,
+                                        _stream(stream)))
+
+
+def forward_host_fp8_async(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, ws_bytes=None,
+                           stream=None):
+    """forward_host_async with FP8 expert weights."""
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    _check("moe_forward_host_fp8_async",
+           lib().moe_forward_host_fp8_async(ctypes.byref(cfg), T, _ptr(x_host), _ptr(W_r), _ptr(b), _fp8(W1),
+                                            _fp8(W3), _fp8(W2), _fp8(Ws1), _fp8(Ws3), _fp8(Ws2), _ptr(y_host),
+                                            _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def host_wait(ws, stream=None) -> None:
+    """Order `stream` after every output copy the asynchronous host calls issued on ws."""
+    _check("moe_host_wait", lib().moe_host_wait(_ptr(ws), _stream(stream)))
+
+
 def workspace_release(ws) -> None:
-    """Free the copy stream and events moe_forward_host keeps for this workspace."""
+    """Free the copy streams and events the host-buffer calls keep for this
+    workspace (blocks until their copies in flight have finished)."""
     _check("moe_workspace_release", lib().moe_workspace_release(_ptr(ws)))
 
 
@@ -354,12 +385,21 @@ class MoELayer:
         fwd(self.cfg, T, x, *self._wargs(), y, self.ws, topk_idx_out, gates_out, stream=stream)
         return y
 
-    def forward_host(self, x_host, y_host, stream=None):
+    def forward_host(self, x_host, y_host, stream=None, wait=True):
+        """x_host in, y_host out (pinned host tensors). With wait=False the
+        output copy runs on the workspace's own stream and overlaps the next
+        call; y_host is then complete after a later host_wait()."""
         T = x_host.shape[0]
         assert T <= self.max_tokens
-        fwd = forward_host_fp8 if self.fp8 else forward_host
+        if wait:
+            fwd = forward_host_fp8 if self.fp8 else forward_host
+        else:
+            fwd = forward_host_fp8_async if self.fp8 else forward_host_async
         fwd(self.cfg, T, x_host, *self._wargs(), y_host, self.ws, stream=stream)
         return y_host
+
+    def host_wait(self, stream=None) -> None:
+        host_wait(self.ws, stream)
 
     def device_status(self, T=None, stream=None) -> int:
         return device_status(self.cfg, self.max_tokens if T is None else T, self.ws, stream=stream)

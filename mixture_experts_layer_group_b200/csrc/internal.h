@@ -43,7 +43,7 @@ struct Problem {
 struct Layout {
   size_t status, sched, logits, idx, gates, chunk_counts, chunk_base, counts, offsets;
   size_t grp_row0, grp_rows, unit_base1, unit_base2, perm, slot_pos, gate_perm;
-  size_t x_perm, h_perm, h_sh, y_rows, x_stage[2], y_stage;
+  size_t x_perm, h_perm, h_sh, y_rows, x_stage[2], y_stage[2];
   size_t total, total_host;
   int64_t n_chunks;
 };

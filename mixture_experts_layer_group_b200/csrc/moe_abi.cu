@@ -147,7 +147,8 @@ Layout make_layout(const Problem& p) {
   L.total = off;
   L.x_stage[0] = take((size_t)T * p.d * p.elem);
   L.x_stage[1] = take((size_t)T * p.d * p.elem);
-  L.y_stage = take((size_t)T * p.d * p.elem);
+  L.y_stage[0] = take((size_t)T * p.d * p.elem);
+  L.y_stage[1] = take((size_t)T * p.d * p.elem);
   L.total_host = off;
   return L;
 }
@@ -271,38 +272,53 @@ moe_status forward_device(const Problem& p, const Layout& L, const void* x, cons
   return MOE_OK;
 }
 
-// Per-workspace state of moe_forward_host: a non-blocking copy stream and
-// a few events (no device memory), created on the workspace's first host
-// call and kept until moe_workspace_release(ws) or the process exits.
+// Per-workspace state of the host-buffer entry points: two non-blocking
+// copy streams (input, output) and a few events (no device memory), created
+// on the workspace's first host call and kept until moe_workspace_release(ws)
+// or the process exits.
 //
-// x is staged in two slots that alternate between calls, so the input copy
-// of one call overlaps the whole of the previous call: the copy into a slot
-// waits only for the end of the call before last (which read that slot).
-// That holds while the workspace layout stays the same; a call with another
-// T or cfg (other offsets, which may overlap regions the previous call still
-// uses), or any device-buffer call on the workspace in between, makes the
-// copy wait for the end of the previous call instead.
+// x and y are each staged in two slots that alternate between calls, so the
+// input copy of one call overlaps the whole of the previous call: the copy
+// into a slot waits only for the end of the call before last (which read
+// that slot). The asynchronous calls copy y out on the output stream, so
+// that copy overlaps the next call too; a call writes a y slot only after
+// the previous copy out of it has finished. That holds while the workspace
+// layout stays the same; a call with another T or cfg (other offsets, which
+// may overlap regions the previous call still uses), or any device-buffer
+// call on the workspace in between, makes the copy wait for the end of the
+// previous call (and its output copy) instead, and every device-buffer call
+// on the workspace first waits for the output copies still pending.
 struct HostPipe {
   int device = -1;
-  cudaStream_t copy = nullptr;
+  cudaStream_t copy = nullptr;      // input copies
+  cudaStream_t out = nullptr;       // output copies of the asynchronous calls
   cudaEvent_t x_ready = nullptr;    // the staged x of the current call has landed
-  cudaEvent_t x_free[2] = {};       // the last call that used slot i no longer reads it
+  cudaEvent_t x_free[2] = {};       // the last call that used x slot i no longer reads it
+  cudaEvent_t y_ready = nullptr;    // the current call's y is in its slot
+  cudaEvent_t y_free[2] = {};       // the last copy out of y slot i has finished
+  cudaEvent_t out_done = nullptr;   // the last asynchronous output copy has finished
   cudaEvent_t done = nullptr;       // end of the last call on this workspace (any entry point)
   bool slot_used[2] = {false, false};
+  bool y_used[2] = {false, false};
+  bool out_pending = false;         // an asynchronous output copy was issued (out_done recorded)
   bool done_recorded = false;
   bool relayout = true;             // next host call must wait for `done`
-  size_t stage_key[3] = {0, 0, 0};  // x slot offsets and bytes of the last host call
+  size_t stage_key[5] = {};         // staging offsets and bytes of the last host call
   uint64_t calls = 0;
 };
 std::mutex g_pipe_mu;
 std::unordered_map<const void*, HostPipe> g_pipes;
 
 void destroy_pipe(HostPipe& hp) {
+  // copies still in flight read or write the caller's buffers: let them end
+  if (hp.copy) cudaStreamSynchronize(hp.copy);
+  if (hp.out) cudaStreamSynchronize(hp.out);
   if (hp.copy) cudaStreamDestroy(hp.copy);
-  if (hp.x_ready) cudaEventDestroy(hp.x_ready);
-  for (int i = 0; i < 2; ++i)
-    if (hp.x_free[i]) cudaEventDestroy(hp.x_free[i]);
-  if (hp.done) cudaEventDestroy(hp.done);
+  if (hp.out) cudaStreamDestroy(hp.out);
+  cudaEvent_t* ev[] = {&hp.x_ready, &hp.x_free[0], &hp.x_free[1], &hp.y_ready, &hp.y_free[0], &hp.y_free[1],
+                       &hp.out_done, &hp.done};
+  for (cudaEvent_t* e : ev)
+    if (*e) cudaEventDestroy(*e);
   hp = HostPipe{};
 }
 
@@ -314,9 +330,11 @@ cudaError_t host_pipe_locked(const void* ws, HostPipe** out) {
   if (hp.device != dev) {
     if (hp.copy) destroy_pipe(hp);  // a different device reuses this address: start over
     e = cudaStreamCreateWithFlags(&hp.copy, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.x_ready, cudaEventDisableTiming);
-    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&hp.x_free[i], cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking);
+    cudaEvent_t* ev[] = {&hp.x_ready, &hp.x_free[0], &hp.x_free[1], &hp.y_ready, &hp.y_free[0], &hp.y_free[1],
+                         &hp.out_done, &hp.done};
+    for (cudaEvent_t* ep : ev)
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ep, cudaEventDisableTiming);
     if (e != cudaSuccess) {
       destroy_pipe(hp);
       return e;
@@ -327,10 +345,20 @@ cudaError_t host_pipe_locked(const void* ws, HostPipe** out) {
   return cudaSuccess;
 }
 
-// A device-buffer entry point (moe_route, moe_dispatch, moe_forward) has
-// enqueued work on `s` that uses ws: if moe_forward_host has state for this
-// workspace, mark the end of that work so the next host call's input copy
-// waits for it (the copy runs on another stream).
+// A device-buffer entry point is about to enqueue work on `s` that uses ws:
+// if asynchronous host calls on this workspace have output copies that may
+// still read it, `s` waits for them first.
+cudaError_t wait_host_outputs(const void* ws, cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  auto it = g_pipes.find(ws);
+  if (it == g_pipes.end() || !it->second.out_pending) return cudaSuccess;
+  return cudaStreamWaitEvent(s, it->second.out_done, 0);
+}
+
+// A device-buffer entry point (moe_route, moe_dispatch, moe_forward, ...) has
+// enqueued work on `s` that uses ws: if the host-buffer calls have state for
+// this workspace, mark the end of that work so the next host call's input
+// copy waits for it (the copy runs on another stream).
 cudaError_t note_device_use(const void* ws, cudaStream_t s) {
   std::lock_guard<std::mutex> lock(g_pipe_mu);
   auto it = g_pipes.find(ws);
@@ -461,43 +489,64 @@ const void* fp8_codes(const Problem& p, const moe_fp8_matrix* const (&m)[6], int
   return (i < 3 || p.ns > 0) ? m[i]->codes : nullptr;
 }
 
-// The host-buffer pipeline of moe_forward_host(_fp8) around one device
-// forward, run(x_device, y_device) on stream s: x is copied into one of the
-// workspace's two staging slots on the workspace's copy stream (overlapping
-// the previous call), y is copied back to the host on s.
+// The host-buffer pipeline of moe_forward_host(_fp8)(_async) around one
+// device forward, run(x_device, y_device) on stream s: x is copied into one
+// of the workspace's two input slots on the input stream (overlapping the
+// previous call); y, written to one of two output slots, is copied back to
+// the host on s, or on the output stream when `async_out` (overlapping the
+// next call).
 template <class Run>
 moe_status forward_host_pipe(const Problem& p, const Layout& L, const void* x_host, void* y_host, void* ws,
-                             cudaStream_t s, Run run) {
+                             cudaStream_t s, bool async_out, Run run) {
   const size_t bytes = (size_t)p.T * p.d * p.elem;
-  void* yd = at<void>(ws, L.y_stage);
   std::lock_guard<std::mutex> lock(g_pipe_mu);
   HostPipe* hp = nullptr;
   cudaError_t e = host_pipe_locked(ws, &hp);
   if (e != cudaSuccess) return cuda_fail(e);
-  const size_t key[3] = {L.x_stage[0], L.x_stage[1], bytes};
+  const size_t key[5] = {L.x_stage[0], L.x_stage[1], L.y_stage[0], L.y_stage[1], bytes};
   if (std::memcmp(key, hp->stage_key, sizeof(key)) != 0) hp->relayout = true;
   if (hp->relayout) {
     // another layout (or device work) since the last host call: the copy may
     // land on regions the previous call still uses, so wait for all of it
     hp->slot_used[0] = hp->slot_used[1] = false;
+    hp->y_used[0] = hp->y_used[1] = false;
     if (hp->done_recorded) e = cudaStreamWaitEvent(hp->copy, hp->done, 0);
+    // and this call's copy and kernels may write where a pending output copy reads
+    if (e == cudaSuccess && hp->out_pending) e = cudaStreamWaitEvent(hp->copy, hp->out_done, 0);
+    if (e == cudaSuccess && hp->out_pending) e = cudaStreamWaitEvent(s, hp->out_done, 0);
     hp->calls = 0;
   }
   const int slot = (int)(hp->calls & 1u);
   void* xd = at<void>(ws, L.x_stage[slot]);
+  void* yd = at<void>(ws, L.y_stage[slot]);
   if (e == cudaSuccess && hp->slot_used[slot]) e = cudaStreamWaitEvent(hp->copy, hp->x_free[slot], 0);
   if (e == cudaSuccess) e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, hp->copy);
   if (e == cudaSuccess) e = cudaEventRecord(hp->x_ready, hp->copy);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->x_ready, 0);
+  // the y slot is written by this call's combine: its last copy out must be over
+  if (e == cudaSuccess && hp->y_used[slot]) e = cudaStreamWaitEvent(s, hp->y_free[slot], 0);
   if (e != cudaSuccess) return cuda_fail(e);
   moe_status st = run(xd, yd);
   if (st != MOE_OK) return st;
-  // the slot is free again once this call's kernels are done
+  // the x slot is free again once this call's kernels are done
   if ((e = cudaEventRecord(hp->x_free[slot], s)) != cudaSuccess) return cuda_fail(e);
   hp->slot_used[slot] = true;
-  e = cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaEventRecord(hp->done, s);
+  if (async_out) {
+    e = cudaEventRecord(hp->y_ready, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->out, hp->y_ready, 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, hp->out);
+    if (e == cudaSuccess) e = cudaEventRecord(hp->y_free[slot], hp->out);
+    if (e == cudaSuccess) e = cudaEventRecord(hp->out_done, hp->out);
+    // the workspace is in use until the output copy ends
+    if (e == cudaSuccess) e = cudaEventRecord(hp->done, hp->out);
+    if (e == cudaSuccess) hp->out_pending = true;
+  } else {
+    e = cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaEventRecord(hp->y_free[slot], s);
+    if (e == cudaSuccess) e = cudaEventRecord(hp->done, s);
+  }
   if (e != cudaSuccess) return cuda_fail(e);
+  hp->y_used[slot] = true;
   hp->done_recorded = true;
   hp->relayout = false;
   std::memcpy(hp->stage_key, key, sizeof(key));
@@ -538,7 +587,8 @@ moe_status moe_route(const moe_cfg* cfg, int64_t T, const void* x, const void* W
   if (!x || !W_r || !topk_idx || !gates || !aligned16(x) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
   Layout L = make_layout(p);
   if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
-  cudaError_t e = cudaMemsetAsync(at<void>(ws, L.status), 0, 4, (cudaStream_t)stream);
+  cudaError_t e = wait_host_outputs(ws, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(at<void>(ws, L.status), 0, 4, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e);
   if ((st = run_router(p, L, x, W_r, b, topk_idx, gates, ws, (cudaStream_t)stream)) != MOE_OK) return st;
   if ((e = note_device_use(ws, (cudaStream_t)stream)) != cudaSuccess) return cuda_fail(e);
@@ -557,7 +607,8 @@ moe_status moe_dispatch(const moe_cfg* cfg, int64_t T, const int32_t* topk_idx, 
   cudaStream_t s = (cudaStream_t)stream;
   DispatchBuffers db = dispatch_buffers(L, ws, topk_idx, nullptr);
   const bool tc = p.dtype == MOE_BF16;
-  cudaError_t e = cudaMemsetAsync(db.status, 0, 4, s);
+  cudaError_t e = wait_host_outputs(ws, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(db.status, 0, 4, s);
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch_dispatch(p, db, tc ? kTcBM : kSimtBM, tc ? kTcBN1 : kSimtBN,
                                   tc ? kTcBN2 : kSimtBN, s);
@@ -585,6 +636,8 @@ moe_status moe_forward(const moe_cfg* cfg, int64_t T, const void* x, const void*
   if ((st = check_weights(p, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2)) != MOE_OK) return st;
   Layout L = make_layout(p);
   if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
+  cudaError_t e0 = wait_host_outputs(ws, (cudaStream_t)stream);
+  if (e0 != cudaSuccess) return cuda_fail(e0);
   st = forward_device(p, L, x, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y, topk_idx_out, gates_out, ws,
                       (cudaStream_t)stream);
   if (st != MOE_OK) return st;
@@ -608,6 +661,8 @@ moe_status moe_forward_fp8(const moe_cfg* cfg, int64_t T, const void* x, const v
   if ((st = check_fp8_ptrs(p, W_r, b, m, &sc)) != MOE_OK) return st;
   Layout L = make_layout(p);
   if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
+  cudaError_t e0 = wait_host_outputs(ws, (cudaStream_t)stream);
+  if (e0 != cudaSuccess) return cuda_fail(e0);
   st = forward_device(p, L, x, W_r, b, fp8_codes(p, m, 0), fp8_codes(p, m, 1), fp8_codes(p, m, 2),
                       fp8_codes(p, m, 3), fp8_codes(p, m, 4), fp8_codes(p, m, 5), y, topk_idx_out, gates_out, ws,
                       (cudaStream_t)stream, &sc);
@@ -616,10 +671,15 @@ moe_status moe_forward_fp8(const moe_cfg* cfg, int64_t T, const void* x, const v
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
-moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
-                            const float* b, const void* W1, const void* W3, const void* W2,
-                            const void* Ws1, const void* Ws3, const void* Ws2, void* y_host,
-                            void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+moe_status forward_host_bf16(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r, const float* b,
+                             const void* W1, const void* W3, const void* W2, const void* Ws1, const void* Ws3,
+                             const void* Ws2, void* y_host, void* ws, size_t ws_bytes, void* stream,
+                             bool async_out) {
   Problem p;
   moe_status st = make_problem(cfg, T, &p);
   if (st != MOE_OK) return st;
@@ -629,16 +689,15 @@ moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, c
   Layout L = make_layout(p);
   if ((st = check_ws(L, ws, ws_bytes, L.total_host)) != MOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  return forward_host_pipe(p, L, x_host, y_host, ws, s, [&](const void* xd, void* yd) {
+  return forward_host_pipe(p, L, x_host, y_host, ws, s, async_out, [&](const void* xd, void* yd) {
     return forward_device(p, L, xd, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, yd, nullptr, nullptr, ws, s);
   });
 }
 
-moe_status moe_forward_host_fp8(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
-                                const float* b, const moe_fp8_matrix* W1, const moe_fp8_matrix* W3,
-                                const moe_fp8_matrix* W2, const moe_fp8_matrix* Ws1, const moe_fp8_matrix* Ws3,
-                                const moe_fp8_matrix* Ws2, void* y_host, void* ws, size_t ws_bytes,
-                                void* stream) {
+moe_status forward_host_fp8(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r, const float* b,
+                            const moe_fp8_matrix* W1, const moe_fp8_matrix* W3, const moe_fp8_matrix* W2,
+                            const moe_fp8_matrix* Ws1, const moe_fp8_matrix* Ws3, const moe_fp8_matrix* Ws2,
+                            void* y_host, void* ws, size_t ws_bytes, void* stream, bool async_out) {
   Problem p;
   moe_status st = make_problem(cfg, T, &p);
   if (st != MOE_OK) return st;
@@ -651,11 +710,51 @@ moe_status moe_forward_host_fp8(const moe_cfg* cfg, int64_t T, const void* x_hos
   Layout L = make_layout(p);
   if ((st = check_ws(L, ws, ws_bytes, L.total_host)) != MOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  return forward_host_pipe(p, L, x_host, y_host, ws, s, [&](const void* xd, void* yd) {
+  return forward_host_pipe(p, L, x_host, y_host, ws, s, async_out, [&](const void* xd, void* yd) {
     return forward_device(p, L, xd, W_r, b, fp8_codes(p, m, 0), fp8_codes(p, m, 1), fp8_codes(p, m, 2),
                           fp8_codes(p, m, 3), fp8_codes(p, m, 4), fp8_codes(p, m, 5), yd, nullptr, nullptr, ws, s,
                           &sc);
   });
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
+                            const float* b, const void* W1, const void* W3, const void* W2,
+                            const void* Ws1, const void* Ws3, const void* Ws2, void* y_host,
+                            void* ws, size_t ws_bytes, void* stream) {
+  return forward_host_bf16(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, ws_bytes, stream, false);
+}
+
+moe_status moe_forward_host_async(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
+                                  const float* b, const void* W1, const void* W3, const void* W2,
+                                  const void* Ws1, const void* Ws3, const void* Ws2, void* y_host,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  return forward_host_bf16(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, ws_bytes, stream, true);
+}
+
+moe_status moe_forward_host_fp8(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
+                                const float* b, const moe_fp8_matrix* W1, const moe_fp8_matrix* W3,
+                                const moe_fp8_matrix* W2, const moe_fp8_matrix* Ws1, const moe_fp8_matrix* Ws3,
+                                const moe_fp8_matrix* Ws2, void* y_host, void* ws, size_t ws_bytes,
+                                void* stream) {
+  return forward_host_fp8(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, ws_bytes, stream, false);
+}
+
+moe_status moe_forward_host_fp8_async(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
+                                      const float* b, const moe_fp8_matrix* W1, const moe_fp8_matrix* W3,
+                                      const moe_fp8_matrix* W2, const moe_fp8_matrix* Ws1,
+                                      const moe_fp8_matrix* Ws3, const moe_fp8_matrix* Ws2, void* y_host,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  return forward_host_fp8(cfg, T, x_host, W_r, b, W1, W3, W2, Ws1, Ws3, Ws2, y_host, ws, ws_bytes, stream, true);
+}
+
+moe_status moe_host_wait(const void* ws, void* stream) {
+  cudaError_t e = wait_host_outputs(ws, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
 moe_status moe_workspace_release(const void* ws) {
@@ -690,7 +789,8 @@ moe_status moe_dispatch_rows(const moe_cfg* cfg, int64_t T, const int32_t* topk_
   db.slot_pos = slot_pos;
   db.gate_perm = gate_perm;
   const bool tc = p.dtype == MOE_BF16;
-  cudaError_t e = cudaMemsetAsync(db.status, 0, 4, s);
+  cudaError_t e = wait_host_outputs(ws, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(db.status, 0, 4, s);
   if (e == cudaSuccess)
     e = launch_dispatch(p, db, tc ? kTcBM : kSimtBM, tc ? kTcBN1 : kSimtBN, tc ? kTcBN2 : kSimtBN, s);
   if (e == cudaSuccess) e = launch_gather(p, x, slot_pos, x_perm, db.status, s);
@@ -722,7 +822,8 @@ moe_status moe_experts(const moe_cfg* cfg, int64_t rows, const int32_t* counts, 
   if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   unsigned* status = at<unsigned>(ws, L.status);
-  cudaError_t e = cudaMemsetAsync(status, 0, 4, s);
+  cudaError_t e = wait_host_outputs(ws, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, 4, s);
   if (e != cudaSuccess) return cuda_fail(e);
   check_counts_kernel<<<1, 256, 0, s>>>(counts, p.N, rows, at<int32_t>(ws, L.counts_in), status);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
@@ -756,6 +857,7 @@ moe_status moe_experts(const moe_cfg* cfg, int64_t rows, const int32_t* counts, 
   ga.status = status;
   ga.sched = at<int>(ws, L.sched);
   e = tc ? launch_expert_gemms_tc(p, ga, s, nullptr) : launch_expert_gemms_simt(p, ga, s, nullptr);
+  if (e == cudaSuccess) e = note_device_use(ws, s);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 

@@ -312,6 +312,75 @@ def test_forward_host_alternating_sizes_and_device_calls():
     moe.workspace_release(ws)
 
 
+def test_forward_host_async_back_to_back_and_mixed_calls():
+    # asynchronous output copies: successive calls on one workspace with no
+    # synchronisation, their y copied out on the workspace's output stream
+    # while the next call runs; mixed with synchronous host calls, other
+    # batch sizes (staging at other offsets) and device-buffer calls (a
+    # moe_forward and a moe_route over a larger batch, whose buffers cover
+    # the staging slots a pending output copy reads). Every y_host must hold
+    # its own batch's output once host_wait has been reached.
+    s = SMALL["v3_like_small"]
+    w = mdev.device_all(s)
+    cfg = cfg_of(s)
+    wargs = (w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"])
+    sizes = [300, 300, 300, 37, 300, 300, 129, 300]
+    big = 600
+    ws = workspace(cfg, big, host=True)
+    xs = [mdev.device_tensor(s.with_(T=T, seed=s.seed + 20 + i), "x") for i, T in enumerate(sizes)]
+    refs = [run_forward(s.with_(T=x.shape[0]), w, x)[0].cpu() for x in xs]
+    xh = [x.cpu().pin_memory() for x in xs]
+    yh = [torch.full_like(h, float("nan")).pin_memory() for h in xh]
+    xd = mdev.device_tensor(s.with_(T=big, seed=98), "x")
+    yd_ref, idx_ref, _ = run_forward(s.with_(T=big), w, xd)
+    yd = torch.empty_like(xd)
+    idx = torch.empty((big, s.top_k), dtype=torch.int32, device="cuda")
+    gates = torch.empty((big, s.top_k), dtype=torch.float32, device="cuda")
+    for rep in range(2):
+        for i, x in enumerate(xh):
+            if i == 5:
+                moe.forward_host(cfg, x.shape[0], x, *wargs, yh[i], ws)  # a synchronous call in between
+            else:
+                moe.forward_host_async(cfg, x.shape[0], x, *wargs, yh[i], ws)
+            if i == 2:
+                moe.forward(cfg, big, xd, *wargs, yd, ws)
+            if i == 6:
+                moe.route(cfg, big, xd, w["W_r"], w["b"], idx, gates, ws)
+        moe.host_wait(ws)
+        torch.cuda.synchronize()
+        for i in range(len(sizes)):
+            assert torch.equal(yh[i], refs[i]), (rep, i)
+            yh[i].fill_(float("nan"))
+        assert torch.equal(yd, yd_ref)
+        assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    # a long run of asynchronous calls of one size, then the wait
+    for rep in range(3):
+        for i in (0, 1, 2, 4):
+            moe.forward_host_async(cfg, 300, xh[i], *wargs, yh[i], ws)
+    moe.host_wait(ws)
+    torch.cuda.synchronize()
+    for i in (0, 1, 2, 4):
+        assert torch.equal(yh[i], refs[i]), i
+    moe.workspace_release(ws)
+
+
+def test_moelayer_async_host_output():
+    s = SMALL["softmax_ragged"]
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    y_dev, _, _ = run_forward(s, w, x)
+    layer = moe.MoELayer(cfg_of(s), w, s.T, host_io=True)
+    xh = x.cpu().pin_memory()
+    yh = [torch.empty_like(xh).pin_memory() for _ in range(3)]
+    for y in yh:
+        layer.forward_host(xh, y, wait=False)
+    layer.host_wait()
+    torch.cuda.synchronize()
+    for y in yh:
+        assert torch.equal(y, y_dev.cpu())
+    moe.workspace_release(layer.ws)
+
+
 def test_abi_errors_on_device_buffers():
     s = SMALL["v3_like_small"]
     cfg = cfg_of(s)
