@@ -186,7 +186,8 @@ def test_fp8_rejects_unsupported_shapes():
 def test_fp8_host_entry_matches_device_entry():
     """moe_forward_host_fp8 (pinned host x in, y out) gives moe_forward_fp8's
     bits, on back-to-back calls that alternate the two staging slots and on a
-    smaller batch on the same workspace afterwards."""
+    smaller batch on the same workspace afterwards; so does
+    moe_forward_host_fp8_async once host_wait has been reached."""
     s = SMALL["fp8_ragged"]
     w = mdev.device_all(s)
     x = mdev.device_tensor(s, "x")
@@ -208,6 +209,15 @@ def test_fp8_host_entry_matches_device_entry():
     torch.cuda.synchronize()
     assert torch.equal(y2h, y2_dev.cpu())
     assert moe.device_status(cfg, T2, ws) == 0
+    # the asynchronous output copies: y_host complete after host_wait
+    for y in yh:
+        y.zero_()
+    for i in range(3):
+        moe.forward_host_fp8_async(cfg, s.T, xh, *wargs, yh[i], ws)
+    moe.host_wait(ws)
+    torch.cuda.synchronize()
+    for i in range(3):
+        assert torch.equal(yh[i], y_dev.cpu())
     moe.workspace_release(ws)
 
 
