@@ -267,11 +267,22 @@ __global__ void __launch_bounds__(256) gather_kernel(const TV* __restrict__ x,
       if (dst[s] >= 0 && !MOE_IN_BOUNDS((int64_t)dst[s] < T * k, status)) dst[s] = -1;
     }
     const TV* src = x + t * vecs;
-    for (int v = v0 + lane; v < v1; v += 32) {
-      const TV val = __ldg(src + v);
+    // two loads in flight per lane before their stores
+    int v = v0 + lane;
+    for (; v + 32 < v1; v += 64) {
+      const TV a = __ldg(src + v), b = __ldg(src + v + 32);
 #pragma unroll
       for (int s = 0; s < KMAX; ++s)
-        if (dst[s] >= 0) x_perm[(int64_t)dst[s] * vecs + v] = val;
+        if (dst[s] >= 0) {
+          x_perm[(int64_t)dst[s] * vecs + v] = a;
+          x_perm[(int64_t)dst[s] * vecs + v + 32] = b;
+        }
+    }
+    if (v < v1) {
+      const TV a = __ldg(src + v);
+#pragma unroll
+      for (int s = 0; s < KMAX; ++s)
+        if (dst[s] >= 0) x_perm[(int64_t)dst[s] * vecs + v] = a;
     }
   }
 }
@@ -369,7 +380,7 @@ cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* slot_p
   const int sms = device_sm_count();
   // warps per token: enough for about 8 warps per SM, at most 8 and at least
   // 32 vectors (one per lane) per part
-  int64_t parts = ((int64_t)sms * 8 + p.T - 1) / p.T;
+  int64_t parts = ((int64_t)sms * 32 + p.T - 1) / p.T;
   if (parts > 8) parts = 8;
   if (parts > vecs / 32) parts = vecs / 32;
   if (parts < 1) parts = 1;
