@@ -119,6 +119,16 @@ SHAPES["v3_prefill_fp8"] = SHAPES["v3_prefill_bf16"].with_(name="v3_prefill_fp8"
 SHAPES["v3_decode_fp8"] = SHAPES["v3_decode_bf16"].with_(name="v3_decode_fp8", wdtype="fp8")
 # The small profiling layer with FP8 weights (1.5 GB of codes: ncu full-section captures)
 SHAPES["v3_profile_32e_fp8"] = SHAPES["v3_profile_32e"].with_(name="v3_profile_32e_fp8", wdtype="fp8")
+# Variants of the V3 prefill layer for DRAM-traffic captures of the expert
+# GEMMs: without the shared expert; without it and without the selection bias
+# (near-uniform routing, no expert over 256 rows); and at half the tokens
+# (no expert over 256 rows either). Same seed, so the same weights and the
+# same leading token rows.
+SHAPES["v3_prefill_noshared_bf16"] = SHAPES["v3_prefill_bf16"].with_(name="v3_prefill_noshared_bf16", n_shared=0)
+SHAPES["v3_prefill_noshared_nobias_bf16"] = SHAPES["v3_prefill_bf16"].with_(
+    name="v3_prefill_noshared_nobias_bf16", n_shared=0, bias=False)
+SHAPES["v3_prefill_t2048_noshared_bf16"] = SHAPES["v3_prefill_bf16"].with_(
+    name="v3_prefill_t2048_noshared_bf16", T=2048, n_shared=0)
 ORDER = ["gshard_tiny_f32", "dsmoe_2b_bf16", "v2_layer_bf16", "v3_prefill_bf16", "v3_decode_bf16"]
 
 
