@@ -1,8 +1,8 @@
 // Dispatch: expert histogram, exclusive scan, expert-contiguous permutation
-// and the row gather that feeds the grouped GEMMs. This replaces the quoted
-// MoE.forward's bincount(...).tolist() and per-expert torch.where loop
-// ("DeepSeek-V3.2-Exp · Mixture of experts", quoted forward excerpt) with
-// three small kernels (one for decode-sized batches) and no host round trip.
+// and the row gather that feeds the grouped GEMMs. The quoted forward of the
+// "DeepSeek-V3.2-Exp · Mixture of experts" page counts the tokens per expert
+// on the host and searches each expert's rows in a loop; here that is three
+// small kernels (one for decode-sized batches) and no host round trip.
 //
 // Bit-exact by construction: a warp owns 32 consecutive tokens; for each
 // expert it forms a ballot of the tokens that chose it, so a pair's rank

@@ -191,8 +191,8 @@ def gates_for(routing_scores: np.ndarray, idx: np.ndarray, cfg: RouterCfg) -> np
 # ------------------------------------------------------------ permutation ----
 
 def permutation(idx: np.ndarray, n_routed: int):
-    """Expert histogram and expert-contiguous token lists, as the excerpt's
-    bincount over the selected indices and its per-expert torch.where:
+    """Expert histogram and expert-contiguous token lists, as the quoted
+    forward counts the selections per expert and finds each expert's rows:
     counts[e] = number of (token, slot) pairs that chose e; offsets is their
     exclusive prefix sum; perm[offsets[e] + r] is the r-th such pair in
     ascending token order, stored as token * k + slot."""
