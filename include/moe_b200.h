@@ -250,8 +250,12 @@ MOE_API moe_status moe_forward_host(const moe_cfg* cfg, int64_t T, const void* x
  * two calls later only after its copy out has finished, and every
  * device-buffer entry point on the workspace (and a host call with another
  * T or cfg) first waits for the output copies still pending, so calls of
- * both kinds can be mixed on one workspace. Same arguments, workspace size
- * and errors as moe_forward_host.
+ * both kinds can be mixed on one workspace. Copies that have finished need
+ * no wait. A CUDA graph capture of device-buffer calls on the workspace may
+ * start once the outputs have been waited for and their stream synchronised,
+ * not while copies are in flight (a capture records no wait on them), and the
+ * caller orders the graph's replays with later host-buffer calls on the same
+ * workspace. Same arguments, workspace size and errors as moe_forward_host.
  */
 MOE_API moe_status moe_forward_host_async(const moe_cfg* cfg, int64_t T, const void* x_host, const void* W_r,
                                           const float* b, const void* W1, const void* W3, const void* W2,

@@ -347,11 +347,24 @@ cudaError_t host_pipe_locked(const void* ws, HostPipe** out) {
 
 // A device-buffer entry point is about to enqueue work on `s` that uses ws:
 // if asynchronous host calls on this workspace have output copies that may
-// still read it, `s` waits for them first.
+// still read it, `s` waits for them first. Copies that have already finished
+// need no wait. A stream under graph capture is not made to wait (and the
+// event is not queried, which a capture forbids): a capture must start only
+// after the outputs have been waited for and their stream synchronised.
 cudaError_t wait_host_outputs(const void* ws, cudaStream_t s) {
   std::lock_guard<std::mutex> lock(g_pipe_mu);
   auto it = g_pipes.find(ws);
   if (it == g_pipes.end() || !it->second.out_pending) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess || cs != cudaStreamCaptureStatusNone) return e;
+  const cudaError_t q = cudaEventQuery(it->second.out_done);
+  if (q == cudaSuccess) {
+    it->second.out_pending = false;
+    return cudaSuccess;
+  }
+  if (q != cudaErrorNotReady) return q;
+  if (cudaPeekAtLastError() == cudaErrorNotReady) (void)cudaGetLastError();  // not an error: drop it
   return cudaStreamWaitEvent(s, it->second.out_done, 0);
 }
 
@@ -364,6 +377,15 @@ cudaError_t note_device_use(const void* ws, cudaStream_t s) {
   auto it = g_pipes.find(ws);
   if (it == g_pipes.end() || !it->second.done) return cudaSuccess;
   it->second.relayout = true;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
+  if (cs != cudaStreamCaptureStatusNone) {
+    // work captured into a graph runs when the graph is launched: the caller
+    // orders its replays with later host-buffer calls on this workspace
+    it->second.done_recorded = false;
+    return cudaSuccess;
+  }
   it->second.done_recorded = true;
   return cudaEventRecord(it->second.done, s);
 }

@@ -364,6 +364,37 @@ def test_forward_host_async_back_to_back_and_mixed_calls():
     moe.workspace_release(ws)
 
 
+def test_graph_capture_after_async_host_calls():
+    # once the asynchronous output copies have finished, a device-buffer
+    # forward on the same workspace captures and replays like on a fresh one
+    s = SMALL["v3_like_small"]
+    w = mdev.device_all(s)
+    x = mdev.device_tensor(s, "x")
+    y_eager, _, _ = run_forward(s, w, x)
+    cfg = cfg_of(s)
+    wargs = (w["W_r"], w["b"], w["W1"], w["W3"], w["W2"], w["Ws1"], w["Ws3"], w["Ws2"])
+    ws = workspace(cfg, s.T, host=True)
+    xh = x.cpu().pin_memory()
+    yh = [torch.empty_like(xh).pin_memory() for _ in range(2)]
+    side = torch.cuda.Stream()
+    for y_h in yh:
+        moe.forward_host_async(cfg, s.T, xh, *wargs, y_h, ws, stream=side)
+    moe.host_wait(ws, side)
+    side.synchronize()
+    for y_h in yh:
+        assert torch.equal(y_h, y_eager.cpu())
+    y = torch.empty_like(x)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        moe.forward(cfg, s.T, x, *wargs, y, ws, stream=side)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_eager)
+    del g
+    moe.workspace_release(ws)
+
+
 def test_moelayer_async_host_output():
     s = SMALL["softmax_ragged"]
     w = mdev.device_all(s)
