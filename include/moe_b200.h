@@ -266,8 +266,10 @@ MOE_API moe_status moe_forward_host_async(const moe_cfg* cfg, int64_t T, const v
  * Makes `stream` wait (on the device, without blocking the host) until every
  * output copy that moe_forward_host_async / moe_forward_host_fp8_async have
  * issued on the workspace at `ws` so far has finished. Returns at once (and
- * MOE_OK) when the workspace has no asynchronous output copies.
- * Errors: MOE_ERR_CUDA from the stream wait.
+ * MOE_OK) when the workspace has no asynchronous output copies or they have
+ * already finished, and records nothing while `stream` is being captured
+ * into a CUDA graph (wait for the copies before the capture starts).
+ * Errors: MOE_ERR_CUDA from the stream query or wait.
  */
 MOE_API moe_status moe_host_wait(const void* ws, void* stream);
 
