@@ -14,7 +14,7 @@ def test_algorithmic_counts_v3_prefill():
     counts = np.full(s.n_routed, s.T * s.top_k // s.n_routed)  # every expert touched
     A = bench.algorithmic(s, counts)
     assert A["U"] == 256
-    # T (k + n_s) 6 d d_ff (the benchmark spec's count)
+    # FLOPs = T (k + n_s) 6 d d_ff: three d x d_ff matrices per selected or shared expert, 2 FLOPs per MAC
     assert A["flops"] == 4096 * 9 * 6 * 7168 * 2048
     # touched expert weights (3 matrices of d x d_ff per expert, bf16) + router + x in + y out
     assert A["layer_bytes"] == 257 * 3 * 7168 * 2048 * 2 + 256 * 7168 * 2 + 2 * 4096 * 7168 * 2
