@@ -1,6 +1,7 @@
 """bench.py host helpers on CPU: the algorithmic FLOP and byte counts the
-roofline fractions divide by, the oracle sample sizing, and the reference
-arm's JSON line on the toy layer."""
+roofline fractions divide by, the oracle sample sizing, the reference arm's
+JSON line on the toy layer, the timed loops' event wait and the clock
+summary."""
 import json
 
 import numpy as np
@@ -49,3 +50,28 @@ def test_reference_arm_line_on_the_toy_layer(capsys):
     assert line["value"] > 0 and line["unit"] == "tokens/s" and line["higher_is_better"] is True
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_wait_event_polls_until_the_event_completes():
+    class FakeEvent:
+        def __init__(self, n):
+            self.left = n
+
+        def query(self):
+            self.left -= 1
+            return self.left < 0
+
+    ev = FakeEvent(3)
+    bench.wait_event(ev, poll_s=0.0)
+    assert ev.left == -1  # queried until it reported completion, and no further
+
+
+def test_clock_summary_counts_throttle_reasons():
+    c = bench.ClockSampler(None)
+    assert c.summary()["reasons"] == ["unsampled"]
+    c.max_mhz = 1965.0
+    c.samples = [(1965.0, 0), (1500.0, 0x4), (1400.0, 0x4 | 0x40)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1500.0 and s["sm_min_mhz"] == 1400.0 and s["samples"] == 3
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert s["reason_samples"] == {"sw_power_cap": 2, "hw_thermal_slowdown": 1}
