@@ -137,6 +137,16 @@ def test_argument_errors_need_no_device(L):
     # shared weights required when n_shared > 0
     assert L.moe_forward(ctypes.byref(cfg), 4, fake, fake, None, fake, fake, fake, None, None, None, fake,
                          None, None, fake, 1 << 40, None) == 1
+    # host-buffer calls: T == 0 is a no-op, null buffers are rejected; waiting on
+    # (or releasing) a workspace without host-call state does nothing
+    for fn in (L.moe_forward_host, L.moe_forward_host_async):
+        assert fn(ctypes.byref(cfg), 0, None, None, None, None, None, None, None, None, None, None, None, 0,
+                  None) == 0
+        assert fn(ctypes.byref(cfg), 4, None, fake, None, fake, fake, fake, fake, fake, fake, fake, fake,
+                  1 << 40, None) == 1
+    assert L.moe_host_wait(None, None) == 0
+    assert L.moe_host_wait(fake, None) == 0
+    assert L.moe_workspace_release(fake) == 0
     # bias update: null / misaligned pointers, non-finite rate
     assert L.moe_bias_update(ctypes.byref(cfg), 4, None, ctypes.c_float(1e-3), fake, None) == 1
     assert L.moe_bias_update(ctypes.byref(cfg), 4, fake, ctypes.c_float(1e-3), fake + 2, None) == 1
